@@ -1,0 +1,173 @@
+"""fp64 CPU oracle for sliding-window attention with a learned per-head sink.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check in
+``__graft_entry__`` and the ``cpu_baseline`` / reference leg of ``bench.py``
+may import this package.  The product library never loads it and has no CPU
+fallback; the two share no code.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision, OpenMP over
+rows); this module only builds it with gcc and marshals numpy arrays.  Inputs
+are passed as bf16 bit patterns (``np.uint16``) so that the oracle reads the
+very bits the device reads.  Each function cites the passage it follows in
+``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP).  No fast-math:
+    the oracle must keep IEEE double semantics."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+             "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        F = ctypes.c_float
+        lib.oracle_num_threads.restype = I
+        lib.oracle_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P]
+        lib.oracle_fwd.restype = I
+        lib.oracle_fwd_rows.argtypes = [P, P, P, P, I, I, I, I, I, I, F, I, P, P, P]
+        lib.oracle_fwd_rows.restype = I
+        lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P]
+        lib.oracle_decode.restype = I
+        lib.oracle_split_partial.argtypes = [P, P, P, ctypes.c_int64, I, I, I, F, P, P]
+        lib.oracle_split_partial.restype = I
+        lib.oracle_combine.argtypes = [I, P, P, I, F, P, P]
+        lib.oracle_combine.restype = I
+        _lib = lib
+    return _lib
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected bf16 bit patterns as uint16, got {a.dtype}")
+    return a
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS or the cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def fwd(q, k, v, sinks, window: int, scale: float, with_lse: bool = True):
+    """Prefill forward (page 1, learned-sink softmax; see oracle.c).
+
+    q [B,L,Hq,D], k/v [B,L,Hkv,D] as uint16 bf16 bits; sinks [Hq] float32.
+    Returns (out [B,L,Hq,D] float64, lse [B,Hq,L] float64 or None)."""
+    q, k, v, sinks = _u16(q), _u16(k), _u16(v), _f32(sinks)
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    assert k.shape == (B, L, Hkv, D) and v.shape == k.shape and sinks.shape == (Hq,)
+    out = np.empty((B, L, Hq, D), np.float64)
+    lse = np.empty((B, Hq, L), np.float64) if with_lse else None
+    rc = _load().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), B, L, Hq, Hkv,
+                            D, int(window), float(scale), _ptr(out),
+                            _ptr(lse) if with_lse else None)
+    if rc != 0:
+        raise ValueError("oracle_fwd: invalid sizes")
+    return out, lse
+
+
+def fwd_rows(q, k, v, sinks, window: int, scale: float, rows):
+    """The forward for selected rows only.  rows: int array [n, 3] of
+    (b, i, h).  Returns (out [n, D] float64, lse [n] float64)."""
+    q, k, v, sinks = _u16(q), _u16(k), _u16(v), _f32(sinks)
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    n = rows.shape[0]
+    out = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), B, L, Hq,
+                                 Hkv, D, int(window), float(scale), n, _ptr(rows),
+                                 _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_fwd_rows: invalid sizes or rows")
+    return out, lse
+
+
+def decode(q, kcache, vcache, seqlens, sinks, window: int, scale: float):
+    """Single-token decode over a contiguous KV cache (see oracle.c).
+
+    q [B,Hq,D]; kcache/vcache [B,Smax,Hkv,D] uint16 bf16 bits; seqlens [B]
+    int32; sinks [Hq] float32.  Returns (out [B,Hq,D], lse [B,Hq]) float64."""
+    q, kcache, vcache, sinks = _u16(q), _u16(kcache), _u16(vcache), _f32(sinks)
+    seqlens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    B, Hq, D = q.shape
+    _, Smax, Hkv, _ = kcache.shape
+    assert kcache.shape == (B, Smax, Hkv, D) and vcache.shape == kcache.shape
+    out = np.empty((B, Hq, D), np.float64)
+    lse = np.empty((B, Hq), np.float64)
+    rc = _load().oracle_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens),
+                               _ptr(sinks), B, Smax, Hq, Hkv, D, int(window),
+                               float(scale), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode: invalid sizes")
+    return out, lse
+
+
+def split_partial(q_row, k_rows, v_rows, lo: int, hi: int, scale: float):
+    """Split-KV step 1 (page 5, section 3): partial softmax of one query row
+    over keys lo..hi (inclusive) of k_rows/v_rows [S, D], no sink.
+    Returns (o_s [D], lse_s)."""
+    q_row, k_rows, v_rows = _u16(q_row), _u16(k_rows), _u16(v_rows)
+    D = q_row.shape[-1]
+    o = np.empty((D,), np.float64)
+    lse = np.empty((1,), np.float64)
+    rc = _load().oracle_split_partial(_ptr(q_row), _ptr(k_rows), _ptr(v_rows),
+                                      k_rows.shape[-1], int(lo), int(hi), D,
+                                      float(scale), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_split_partial: invalid range")
+    return o, float(lse[0])
+
+
+def combine(lse_s, o_s, sink: float):
+    """Split-KV step 2 (page 5, section 3): log-sum-exp merge of the splits
+    that exist, in order, with the sink once.  lse_s [n], o_s [n, D].
+    Returns (out [D], lse)."""
+    lse_s = np.ascontiguousarray(np.asarray(lse_s, dtype=np.float64))
+    o_s = np.ascontiguousarray(np.asarray(o_s, dtype=np.float64))
+    n = lse_s.shape[0]
+    D = o_s.shape[-1]
+    out = np.empty((D,), np.float64)
+    lse = np.empty((1,), np.float64)
+    rc = _load().oracle_combine(n, _ptr(lse_s), _ptr(o_s), D, float(sink),
+                                _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_combine: invalid sizes")
+    return out, float(lse[0])
