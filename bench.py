@@ -1,0 +1,408 @@
+"""Benchmark of the hot path: prefill forward + split-KV decode.
+
+One step = one attn_sink_fwd over the prefill workload (B2 Hq32 Hkv4 L4096
+D128 W513) followed by one attn_sink_decode over the decode workload (B64
+Hq32 Hkv4 D128, lengths ~ U[4096, 131072]), both on synthetic seeded inputs
+already resident in HBM.  Between steps a 256 MB buffer is written to flush
+L2 (the prefill inputs are smaller than L2; the decode cache is ~17 GB).
+
+`value` is useful prefill TFLOP/s (window-visible pairs only), summed over
+ranks, from CUDA events around each prefill launch; the decode figure (HBM
+GB/s of algorithmic bytes) is reported beside it.  `--impl reference` times
+the fp64 CPU oracle on a bounded sample of the same prefill workload.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+(N > 1: launch under torchrun; each rank runs its own copy of the workloads.)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sliding_window_learned_b200 import inputs  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s (useful) & % bf16 tensor peak; decode HBM GB/s & % of peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def useful_fwd_flops(cfg) -> float:
+    """4*D per visible (query, key) pair: QK^T and PV, window-visible pairs only."""
+    L, W = cfg.L, cfg.W
+    i = np.arange(L, dtype=np.int64)
+    pairs = int(np.minimum(i + 1, W).sum())
+    return 4.0 * cfg.D * cfg.B * cfg.Hq * pairs
+
+
+def decode_bytes(cfg, seqlens) -> float:
+    """K and V rows of the visible keys of every (sequence, kv head), plus q and out."""
+    n = np.asarray(seqlens, dtype=np.int64)
+    vis = n - np.maximum(0, n - cfg.W)
+    kv = int(vis.sum()) * cfg.Hkv * cfg.D * 2 * 2
+    return float(kv + 2 * cfg.B * cfg.Hq * cfg.D * 2)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic(kernel: str, sources: list[str]):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    h = hashlib.sha256()
+    for s in sources:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != d.get("src_sha256"):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.idx = device_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import sliding_window_learned_b200 as swl
+    from sliding_window_learned_b200 import build as swl_build
+
+    if rank == 0:
+        swl_build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- workloads (per rank; weak scaling) ----
+    pcfg, dcfg = inputs.PREFILL, inputs.DECODE
+    x = inputs.make_prefill(pcfg, seed=rank)
+    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    sinks = x["sinks"].to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(pcfg.B, pcfg.Hq, pcfg.L, dtype=torch.float32, device=dev)
+    y = inputs.make_decode(dcfg, seed=rank, device=dev)
+    dout = torch.empty_like(y["q"])
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    fwd_flops = useful_fwd_flops(pcfg)
+    dbytes = decode_bytes(dcfg, y["seqlens"].cpu().numpy())
+
+    def fwd():
+        swl.attn_sink_fwd(q, k, v, sinks, pcfg.W, pcfg.scale, out, lse, stream)
+
+    def dec():
+        swl.attn_sink_decode(y["q"], y["kcache"], y["vcache"], y["seqlens"], y["sinks"], dcfg.W,
+                             dcfg.scale, dout, stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1.0)
+        fwd()
+        dec()
+    torch.cuda.synchronize()
+    if swl.attn_sink_get_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    ev_all = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ev_all[0].record(stream)
+    for s in range(K):
+        flush.fill_(1.0)
+        ev[s][0].record(stream)
+        fwd()
+        ev[s][1].record(stream)
+        ev[s][2].record(stream)
+        dec()
+        ev[s][3].record(stream)
+    ev_all[1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    if swl.attn_sink_get_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+    t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3       # s, K launches
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    t_all = ev_all[0].elapsed_time(ev_all[1]) / 1e3
+
+    # ---- end to end through the public API: pinned host -> device -> host ----
+    hq, hk, hv = x["q"].pin_memory(), x["k"].pin_memory(), x["v"].pin_memory()
+    hs = x["sinks"].pin_memory()
+    ho, hl = torch.empty_like(hq).pin_memory(), torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    Ke = max(3, min(K, 20))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        sinks.copy_(hs, non_blocking=True)
+        fwd()
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) / 1e3
+
+    # ---- max over ranks ----
+    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    t_fwd, t_dec, t_all, t_e2e = times.tolist()
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fwd_tflops = world * K * fwd_flops / t_fwd / 1e12
+    per_launch_fwd = t_fwd / K
+    per_launch_dec = t_dec / K
+    achieved_fwd = fwd_flops / per_launch_fwd / 1e12
+    achieved_dec = dbytes / per_launch_dec / 1e9
+    dec_gbs = world * K * dbytes / t_dec / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(fwd_tflops, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round((t_fwd + t_dec) / K * 1e3, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; torch generator, seed = rank)",
+        "config": {"workload": inputs.PREFILL.name, "decode_workload": inputs.DECODE.name,
+                   "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MB write)"},
+        "roofline": {"kernel": "fwd_tc_kernel<128,128>", "bound": "tensor",
+                     "achieved": round(achieved_fwd, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved_fwd / bf16_peak, 4),
+                     "peak_source": f"{peak_src} bf16 (burst)",
+                     "traffic": profiled_traffic("fwd_tc", ["sliding_window_learned_b200/csrc/fwd_tc.cu",
+                                                            "sliding_window_learned_b200/csrc/ptx.cuh"]),
+                     "flops_per_launch": fwd_flops, "ms_per_launch": round(per_launch_fwd * 1e3, 5)},
+        "decode": {"value": round(dec_gbs, 2), "unit": "GB/s", "ms_per_call": round(per_launch_dec * 1e3, 4),
+                   "bytes_per_call": dbytes,
+                   "roofline": {"kernel": "plan + split + combine", "bound": "hbm",
+                                "achieved": round(achieved_dec, 2), "peak": hbm_peak, "unit": "GB/s",
+                                "frac": round(achieved_dec / hbm_peak, 4),
+                                "peak_source": f"{peak_src} copy bandwidth",
+                                "traffic": profiled_traffic("decode_split", [
+                                    "sliding_window_learned_b200/csrc/decode.cu",
+                                    "sliding_window_learned_b200/csrc/ptx.cuh"])}},
+        "e2e": {"value": round(world * Ke * fwd_flops / t_e2e / 1e12, 4), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "attn_sink_fwd with pinned host inputs copied in and O, LSE copied out each step"},
+        "gpu_launches": K * 4,
+        "clocks": clk,
+        "timed_region_ms": round(t_all * 1e3, 3),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------- oracle timing
+_PREFILL_HOST = {}
+
+
+def _oracle_sample(n_rows, seed=0):
+    cfg = inputs.PREFILL
+    if "x" not in _PREFILL_HOST:
+        _PREFILL_HOST["x"] = inputs.make_prefill(cfg, seed=0)
+    x = _PREFILL_HOST["x"]
+    rng = np.random.default_rng(seed)
+    rows = np.stack([rng.integers(cfg.B, size=n_rows), rng.integers(cfg.L, size=n_rows),
+                     rng.integers(cfg.Hq, size=n_rows)], 1).astype(np.int32)
+    vis = np.minimum(rows[:, 1].astype(np.int64) + 1, cfg.W)
+    flops = 4.0 * cfg.D * float(vis.sum())
+    import oracle
+    if "bits" not in _PREFILL_HOST:
+        _PREFILL_HOST["bits"] = (inputs.bits(x["q"]), inputs.bits(x["k"]), inputs.bits(x["v"]))
+    qb, kb, vb = _PREFILL_HOST["bits"]
+    sk = x["sinks"].numpy()
+
+    def run():
+        oracle.fwd_rows(qb, kb, vb, sk, cfg.W, cfg.scale, rows)
+
+    return run, flops
+
+
+def cpu_baseline(budget_s: float = 10.0):
+    """The fp64 oracle, as it stands, on a bounded random sample of rows of the
+    prefill workload; useful TFLOP/s of the sampled rows."""
+    import oracle
+    oracle.build()
+    run, flops = _oracle_sample(256)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    n_rows = int(max(256, min(200000, 256 * budget_s / max(dt, 1e-6))))
+    run, flops = _oracle_sample(n_rows, seed=1)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n_rows} random (b, i, h) rows of {inputs.PREFILL.name}, fp64, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    run, flops = _oracle_sample(256)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    # each step a bounded sample: the whole run stays within ~2 minutes
+    budget_per_step = min(20.0, 120.0 / max(1, args.steps + args.warmup))
+    n_rows = int(max(64, min(100000, 256 * budget_per_step / max(dt, 1e-6))))
+    steps = []
+    for s in range(args.warmup + args.steps):
+        run, flops = _oracle_sample(n_rows, seed=100 + s)
+        t0 = time.perf_counter()
+        run()
+        if s >= args.warmup:
+            steps.append((flops, time.perf_counter() - t0))
+    fl = sum(f for f, _ in steps)
+    tt = sum(t for _, t in steps)
+    value = fl / tt / 1e12
+    sample = f"{n_rows} random (b, i, h) rows of {inputs.PREFILL.name} per step, fp64"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tt / max(1, len(steps)) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; torch generator, seed 0)",
+        "config": {"workload": inputs.PREFILL.name, "parallelism": "cpu"},
+        "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "sample": sample,
+                         "value": round(value, 6), "unit": "TFLOP/s"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

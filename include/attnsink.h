@@ -1,0 +1,158 @@
+/*
+ * attnsink.h -- C ABI of libattnsink.so: exact causal sliding-window attention
+ * with one learned sink logit per head, and its split-KV decode, for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operation (page "cf-1.com/news/6055759", section "why it must change:
+ * Flint's learned sink"): every query attends to the W most recent keys of its
+ * sequence, itself included, and a per-head scalar sink logit joins the softmax
+ * denominator as a virtual anchor without a value row.  For query row i of
+ * head h, with kv head hk = h / (Hq/Hkv) and visible keys
+ * V(i) = { j : max(0, i-W+1) <= j <= i }:
+ *
+ *   s_j   = scale * <q_i, k_j>
+ *   O_i   = sum_{j in V(i)} e^{s_j} v_j / ( sum_{j in V(i)} e^{s_j} + e^{sink_h} )
+ *   LSE_i = ln( sum_{j in V(i)} e^{s_j} + e^{sink_h} )
+ *
+ * The sink is in logit units after scaling (it is not multiplied by scale).
+ * Same page, section "fix 2: sink normalisation": the kernels rebase the running
+ * maximum on the sink so that no exponent is positive, whichever side dominates.
+ *
+ * Conventions for every entry point:
+ *  - All tensors are described by attn_tensor: a DEVICE pointer, a dtype, and
+ *    shape/stride in elements.  The innermost dimension must have stride 1;
+ *    every other stride of a bf16 tensor must be a positive multiple of 8
+ *    elements (16 bytes) and every base pointer 16-byte aligned.
+ *  - The caller owns every buffer.  The library keeps no pointer after a call
+ *    returns.  Launches go to `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and are stream-ordered: no call synchronises the host.
+ *  - Calls never abort.  They return ATTN_OK or a negative attn_status code.
+ *    Argument errors are detected on the host before anything is launched; a
+ *    one-line description of the last error on the calling thread is available
+ *    from attn_sink_last_error().
+ *  - Device-side waits are bounded.  A wait that runs out records
+ *    ATTN_ETIMEOUT in a device status word and the kernel returns early;
+ *    attn_sink_get_status() reads and clears that word.
+ */
+#ifndef ATTNSINK_H
+#define ATTNSINK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum attn_dtype {
+    ATTN_DTYPE_BF16 = 1,
+    ATTN_DTYPE_F32 = 2,
+    ATTN_DTYPE_I32 = 3
+};
+
+typedef struct attn_tensor {
+    void *data;        /* device pointer (16-byte aligned)                  */
+    int32_t dtype;     /* enum attn_dtype                                    */
+    int32_t ndim;      /* number of valid entries in shape/stride            */
+    int64_t shape[4];
+    int64_t stride[4]; /* in elements                                        */
+} attn_tensor;
+
+enum attn_status {
+    ATTN_OK = 0,
+    ATTN_EINVAL = -1,       /* bad shape, dtype, stride, alignment or value   */
+    ATTN_EUNSUPPORTED = -2, /* valid but not implemented (e.g. head dim)      */
+    ATTN_ECUDA = -3,        /* a CUDA runtime call failed                     */
+    ATTN_ENOMEM = -4,       /* stream-ordered workspace allocation failed     */
+    ATTN_ETIMEOUT = -5      /* a device-side bounded wait ran out             */
+};
+
+/*
+ * Prefill forward (page "cf-1.com/news/6055759": learned sink, fix 2).
+ *
+ *   q      [B, L, Hq, D]  bf16
+ *   k, v   [B, L, Hkv, D] bf16, Hq % Hkv == 0
+ *   sinks  [Hq]           f32; finite or -inf (-inf = no sink).  +inf or NaN
+ *                         give an undefined result.
+ *   window W >= 1: number of visible keys including the query's own position;
+ *          any W >= L is full causal attention.
+ *   scale  softmax scale applied to q.k (typically 1/sqrt(D)); finite, > 0.
+ *   out    [B, L, Hq, D]  bf16, written completely (round to nearest even).
+ *   lse    [B, Hq, L]     f32 natural-log normaliser including the sink, or
+ *                         NULL.  The innermost stride must be 1.
+ * Supported head dims D: 64, 128, 256.  L = 0 or B = 0 is a no-op.
+ * Runs on the tcgen05/TMEM tensor-core kernel.
+ */
+int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                  const attn_tensor *sinks, int32_t window, float scale,
+                  attn_tensor *out, attn_tensor *lse, void *stream);
+
+/*
+ * The same operation on a plain CUDA-core fp32 kernel (one warp per output
+ * row).  Slow; it is an independent second implementation for verification
+ * and debugging, with the same arguments and semantics as attn_sink_fwd, and
+ * any D that is a multiple of 32 up to 256.
+ */
+int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k,
+                           const attn_tensor *v, const attn_tensor *sinks,
+                           int32_t window, float scale, attn_tensor *out,
+                           attn_tensor *lse, void *stream);
+
+/*
+ * Single-token split-KV decode over a contiguous KV cache (page
+ * "flashmla-optimization/docs/PATCH_STACK.md", section 3 "exact small-split
+ * combine"; split-KV decode benchmark on the flash-attention contributor
+ * guide page).
+ *
+ *   q        [B, Hq, D]       bf16; the query of sequence b sits at position
+ *                             seqlens[b]-1 and its own key/value are already
+ *                             in the cache.
+ *   kcache,
+ *   vcache   [B, Smax, Hkv, D] bf16; only positions < seqlens[b] are read.
+ *   seqlens  [B] int32, DEVICE memory, 0 <= seqlens[b] <= Smax (values outside
+ *            are clamped; a sequence of length 0 yields a zero output row).
+ *   sinks    [Hq] f32, as for attn_sink_fwd.
+ *   window   visible keys are [max(0, n-W), n-1] for n = seqlens[b].
+ *   out      [B, Hq, D] bf16.
+ *
+ * Three launches on `stream`, no host synchronisation: a planner reads the
+ * lengths on the device and splits each sequence's visible range into chunks;
+ * a split kernel writes one partial (O_s, LSE_s) per (sequence, head, chunk);
+ * a combine kernel merges only the chunks that exist, in chunk order, adding
+ * the sink once.  The partials live in a workspace taken from a library-owned
+ * stream-ordered memory pool (cudaMallocAsync/cudaFreeAsync on `stream`).
+ * Supported: D in {64, 128, 256}, Hq/Hkv <= 16.
+ */
+int attn_sink_decode(const attn_tensor *q, const attn_tensor *kcache,
+                     const attn_tensor *vcache, const attn_tensor *seqlens,
+                     const attn_tensor *sinks, int32_t window, float scale,
+                     attn_tensor *out, void *stream);
+
+/*
+ * attn_sink_decode with an explicit split size: `chunk` keys per split
+ * (a positive multiple of 64, or 0 for the library's choice, which keeps every
+ * sequence at <= 32 splits).  Used to force a given number of splits.
+ */
+int attn_sink_decode_chunked(const attn_tensor *q, const attn_tensor *kcache,
+                             const attn_tensor *vcache, const attn_tensor *seqlens,
+                             const attn_tensor *sinks, int32_t window, float scale,
+                             int32_t chunk, attn_tensor *out, void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the
+ * current device: ATTN_OK, ATTN_ETIMEOUT (a bounded wait ran out), or
+ * ATTN_ECUDA if the synchronisation itself failed.
+ */
+int attn_sink_get_status(void *stream);
+
+/* Static description of an attn_status code. */
+const char *attn_sink_strerror(int code);
+
+/* One-line description of the last error returned on the calling thread
+ * (empty string if none).  Valid until the next call on that thread. */
+const char *attn_sink_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTNSINK_H */

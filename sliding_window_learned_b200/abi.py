@@ -1,0 +1,190 @@
+"""ctypes binding of libattnsink.so (C ABI declared in include/attnsink.h).
+
+Argument marshalling only: torch tensors are described as ``attn_tensor``
+structs (device pointer, dtype, shape, strides) and passed to the library,
+which runs every step on the GPU.  There is no CPU fallback: if the library
+is missing or a call fails, an exception is raised.
+
+The functions carry the C names.  ``stream`` defaults to torch's current CUDA
+stream on the tensors' device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattnsink.so")
+
+ATTN_OK = 0
+ATTN_EINVAL = -1
+ATTN_EUNSUPPORTED = -2
+ATTN_ECUDA = -3
+ATTN_ENOMEM = -4
+ATTN_ETIMEOUT = -5
+
+ATTN_DTYPE_BF16 = 1
+ATTN_DTYPE_F32 = 2
+ATTN_DTYPE_I32 = 3
+
+_DTYPES = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float32: ATTN_DTYPE_F32,
+           torch.int32: ATTN_DTYPE_I32}
+
+# Every symbol include/attnsink.h declares.
+EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_cudacore", "attn_sink_decode",
+           "attn_sink_decode_chunked", "attn_sink_get_status", "attn_sink_strerror",
+           "attn_sink_last_error")
+
+
+class AttnTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class AttnSinkError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str):
+        self.code = code
+        super().__init__(f"{where}: {detail or 'error'} (code {code})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libattnsink.so (built by ``python -m sliding_window_learned_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libattnsink.so is not built ({LIB_PATH}); run "
+                              "`python -m sliding_window_learned_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(AttnTensor)
+        V = ctypes.c_void_p
+        i32, f32 = ctypes.c_int32, ctypes.c_float
+        for name in ("attn_sink_fwd", "attn_sink_fwd_cudacore"):
+            fn = getattr(lib, name)
+            fn.argtypes = [P, P, P, P, i32, f32, P, P, V]
+            fn.restype = ctypes.c_int
+        lib.attn_sink_decode.argtypes = [P, P, P, P, P, i32, f32, P, V]
+        lib.attn_sink_decode.restype = ctypes.c_int
+        lib.attn_sink_decode_chunked.argtypes = [P, P, P, P, P, i32, f32, i32, P, V]
+        lib.attn_sink_decode_chunked.restype = ctypes.c_int
+        lib.attn_sink_get_status.argtypes = [V]
+        lib.attn_sink_get_status.restype = ctypes.c_int
+        lib.attn_sink_strerror.argtypes = [ctypes.c_int]
+        lib.attn_sink_strerror.restype = ctypes.c_char_p
+        lib.attn_sink_last_error.argtypes = []
+        lib.attn_sink_last_error.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def describe(t: torch.Tensor | None):
+    """An attn_tensor describing a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    if t.dim() > 4:
+        raise ValueError("at most 4 dimensions")
+    d = AttnTensor()
+    d.data = t.data_ptr() if t.numel() > 0 else None
+    d.dtype = _DTYPES[t.dtype]
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _ref(d):
+    return ctypes.byref(d) if d is not None else None
+
+
+def _stream(stream, t: torch.Tensor):
+    if stream is None:
+        return torch.cuda.current_stream(t.device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc: int, where: str):
+    if rc != ATTN_OK:
+        detail = load().attn_sink_last_error().decode()
+        raise AttnSinkError(rc, where, detail)
+
+
+def attn_sink_fwd(q, k, v, sinks, window: int, scale: float, out, lse=None, stream=None):
+    """C ``attn_sink_fwd``: tcgen05 prefill forward into ``out`` (and ``lse``)."""
+    lib = load()
+    ds = [describe(x) for x in (q, k, v, sinks, out, lse)]
+    rc = lib.attn_sink_fwd(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), int(window),
+                           float(scale), _ref(ds[4]), _ref(ds[5]), _stream(stream, q))
+    _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_fwd_cudacore(q, k, v, sinks, window: int, scale: float, out, lse=None, stream=None):
+    """C ``attn_sink_fwd_cudacore``: the CUDA-core fp32 second implementation."""
+    lib = load()
+    ds = [describe(x) for x in (q, k, v, sinks, out, lse)]
+    rc = lib.attn_sink_fwd_cudacore(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]),
+                                    int(window), float(scale), _ref(ds[4]), _ref(ds[5]),
+                                    _stream(stream, q))
+    _check(rc, "attn_sink_fwd_cudacore")
+
+
+def attn_sink_decode(q, kcache, vcache, seqlens, sinks, window: int, scale: float, out,
+                     stream=None):
+    """C ``attn_sink_decode``: split-KV decode into ``out``."""
+    lib = load()
+    ds = [describe(x) for x in (q, kcache, vcache, seqlens, sinks, out)]
+    rc = lib.attn_sink_decode(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), _ref(ds[4]),
+                              int(window), float(scale), _ref(ds[5]), _stream(stream, q))
+    _check(rc, "attn_sink_decode")
+
+
+def attn_sink_decode_chunked(q, kcache, vcache, seqlens, sinks, window: int, scale: float,
+                             chunk: int, out, stream=None):
+    """C ``attn_sink_decode_chunked``: split-KV decode with ``chunk`` keys per split."""
+    lib = load()
+    ds = [describe(x) for x in (q, kcache, vcache, seqlens, sinks, out)]
+    rc = lib.attn_sink_decode_chunked(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]),
+                                      _ref(ds[4]), int(window), float(scale), int(chunk),
+                                      _ref(ds[5]), _stream(stream, q))
+    _check(rc, "attn_sink_decode_chunked")
+
+
+def attn_sink_get_status(stream=None) -> int:
+    """C ``attn_sink_get_status``: sync ``stream`` and read/clear the device status."""
+    lib = load()
+    s = stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else stream
+    return int(lib.attn_sink_get_status(s))
+
+
+def attn_sink_strerror(code: int) -> str:
+    return load().attn_sink_strerror(int(code)).decode()
+
+
+def attn_sink_last_error() -> str:
+    return load().attn_sink_last_error().decode()
+
+
+# ---------------------------------------------------------------- conveniences
+def fwd(q, k, v, sinks, window: int, scale: float, with_lse: bool = True, stream=None):
+    """Allocate outputs and run attn_sink_fwd.  Returns (out, lse or None)."""
+    B, L, Hq, D = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device) if with_lse else None
+    attn_sink_fwd(q, k, v, sinks, window, scale, out, lse, stream)
+    return out, lse
+
+
+def decode(q, kcache, vcache, seqlens, sinks, window: int, scale: float, chunk: int = 0,
+           stream=None):
+    """Allocate the output and run the split-KV decode.  Returns out [B,Hq,D]."""
+    out = torch.empty_like(q)
+    attn_sink_decode_chunked(q, kcache, vcache, seqlens, sinks, window, scale, chunk, out, stream)
+    return out

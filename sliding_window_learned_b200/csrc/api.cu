@@ -1,0 +1,370 @@
+// api.cu -- the C ABI of libattnsink.so (declared in include/attnsink.h):
+// argument validation, the device status word, the decode workspace pool and
+// TMA descriptor encoding.  Every compute step runs in the kernels; nothing
+// here touches tensor data on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/attnsink.h"
+#include "kernels.h"
+
+namespace attnsink {
+
+// Device status word: [0] = first error code, [1] = location of the failing
+// wait.  Kernels receive its address; attn_sink_get_status reads and clears it.
+__device__ int g_status[2];
+
+namespace {
+
+thread_local char t_last_error[256] = "";
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int fail_cuda(cudaError_t e, const char *what) {
+  return fail(e == cudaErrorMemoryAllocation ? ATTN_ENOMEM : ATTN_ECUDA, "%s: %s", what,
+              cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int *g_status_ptr[kMaxDevices];
+cudaMemPool_t g_pool[kMaxDevices];
+bool g_pool_ready[kMaxDevices];
+
+int current_device(int *dev) {
+  const cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(ATTN_EUNSUPPORTED, "device index %d", *dev);
+  return ATTN_OK;
+}
+
+int status_ptr(int **out) {
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_status);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(status)");
+    g_status_ptr[dev] = static_cast<int *>(p);
+  }
+  *out = g_status_ptr[dev];
+  return ATTN_OK;
+}
+
+// A private stream-ordered pool per device that keeps freed blocks cached, so
+// repeated decode calls reuse their workspace without new mappings.
+int workspace_pool(cudaMemPool_t *out) {
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_pool_ready[dev]) {
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof props);
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaError_t e = cudaMemPoolCreate(&g_pool[dev], &props);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemPoolSetAttribute");
+    g_pool_ready[dev] = true;
+  }
+  *out = g_pool[dev];
+  return ATTN_OK;
+}
+
+// ------------------------------------------------------------ validation
+const char *dtype_name(int32_t d) {
+  switch (d) {
+    case ATTN_DTYPE_BF16: return "bf16";
+    case ATTN_DTYPE_F32: return "f32";
+    case ATTN_DTYPE_I32: return "i32";
+    default: return "unknown";
+  }
+}
+
+int check_tensor(const attn_tensor *t, const char *name, int32_t dtype, int ndim, bool tma) {
+  if (!t) return fail(ATTN_EINVAL, "%s: null tensor", name);
+  if (t->dtype != dtype)
+    return fail(ATTN_EINVAL, "%s: dtype %s, expected %s", name, dtype_name(t->dtype), dtype_name(dtype));
+  if (t->ndim != ndim) return fail(ATTN_EINVAL, "%s: ndim %d, expected %d", name, t->ndim, ndim);
+  int64_t numel = 1;
+  for (int d = 0; d < ndim; ++d) {
+    if (t->shape[d] < 0) return fail(ATTN_EINVAL, "%s: negative size in dim %d", name, d);
+    numel *= t->shape[d];
+  }
+  if (numel > 0 && !t->data) return fail(ATTN_EINVAL, "%s: null data pointer", name);
+  if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0)
+    return fail(ATTN_EINVAL, "%s: data pointer not 16-byte aligned", name);
+  if (t->stride[ndim - 1] != 1 && t->shape[ndim - 1] > 1)
+    return fail(ATTN_EINVAL, "%s: innermost stride must be 1", name);
+  for (int d = 0; d < ndim - 1; ++d) {
+    if (t->stride[d] <= 0) return fail(ATTN_EINVAL, "%s: stride of dim %d must be positive", name, d);
+    if (tma && t->stride[d] % 8 != 0)
+      return fail(ATTN_EINVAL, "%s: stride of dim %d must be a multiple of 8 elements", name, d);
+  }
+  return ATTN_OK;
+}
+
+bool finite_pos(float x) { return isfinite(x) && x > 0.f; }
+
+int prep_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+             const attn_tensor *sinks, int32_t window, float scale, attn_tensor *out,
+             attn_tensor *lse, bool tma, FwdArgs *a) {
+  int rc;
+  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 4, tma))) return rc;
+  if ((rc = check_tensor(k, "k", ATTN_DTYPE_BF16, 4, tma))) return rc;
+  if ((rc = check_tensor(v, "v", ATTN_DTYPE_BF16, 4, tma))) return rc;
+  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(out, "out", ATTN_DTYPE_BF16, 4, tma))) return rc;
+  const int64_t B = q->shape[0], L = q->shape[1], Hq = q->shape[2], D = q->shape[3];
+  const int64_t Hkv = k->shape[2];
+  if (k->shape[0] != B || k->shape[1] != L || k->shape[3] != D)
+    return fail(ATTN_EINVAL, "k shape does not match q");
+  for (int d = 0; d < 4; ++d)
+    if (v->shape[d] != k->shape[d]) return fail(ATTN_EINVAL, "v shape does not match k");
+  for (int d = 0; d < 4; ++d)
+    if (out->shape[d] != q->shape[d]) return fail(ATTN_EINVAL, "out shape does not match q");
+  if (sinks->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks must have Hq = %lld entries", (long long)Hq);
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
+  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
+  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
+  if (lse) {
+    if ((rc = check_tensor(lse, "lse", ATTN_DTYPE_F32, 3, false))) return rc;
+    if (lse->shape[0] != B || lse->shape[1] != Hq || lse->shape[2] != L)
+      return fail(ATTN_EINVAL, "lse must be [B, Hq, L]");
+  }
+  if (B > 65535 || Hq > 65535 || L > (1LL << 30))
+    return fail(ATTN_EUNSUPPORTED, "B and Hq must be <= 65535 and L <= 2^30");
+  a->q = q->data;
+  a->k = k->data;
+  a->v = v->data;
+  a->sinks = static_cast<const float *>(sinks->data);
+  a->out = out->data;
+  a->lse = lse ? static_cast<float *>(lse->data) : nullptr;
+  a->B = static_cast<int>(B);
+  a->L = static_cast<int>(L);
+  a->Hq = static_cast<int>(Hq);
+  a->Hkv = static_cast<int>(Hkv);
+  a->D = static_cast<int>(D);
+  a->W = window;
+  a->scale = scale;
+  for (int d = 0; d < 3; ++d) {
+    a->q_s[d] = q->stride[d];
+    a->k_s[d] = k->stride[d];
+    a->v_s[d] = v->stride[d];
+    a->o_s[d] = out->stride[d];
+  }
+  a->lse_s[0] = lse ? lse->stride[0] : 0;
+  a->lse_s[1] = lse ? lse->stride[1] : 0;
+  if (sinks->shape[0] > 1 && sinks->stride[0] != 1) return fail(ATTN_EINVAL, "sinks must be contiguous");
+  return ATTN_OK;
+}
+
+}  // namespace
+
+// TMA descriptor for a [d3, d2, d1, d0] bf16 tensor, box {64, 1, box_rows, 1},
+// 128-byte swizzle, zero fill out of range.
+cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
+                          int64_t d0, const int64_t strides_el[3], int box_rows) {
+  typedef CUresult (*encode_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static encode_fn encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<encode_fn>(fn);
+  });
+  if (!encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
+                              static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
+  // byte strides of dims 1..3 (innermost first): head, position, batch
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(strides_el[2]) * 2,
+                                 static_cast<cuuint64_t>(strides_el[1]) * 2,
+                                 static_cast<cuuint64_t>(strides_el[0]) * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = encode(static_cast<CUtensorMap *>(map_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                            const_cast<void *>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace attnsink
+
+using namespace attnsink;
+
+extern "C" {
+
+const char *attn_sink_strerror(int code) {
+  switch (code) {
+    case ATTN_OK: return "success";
+    case ATTN_EINVAL: return "invalid argument";
+    case ATTN_EUNSUPPORTED: return "unsupported configuration";
+    case ATTN_ECUDA: return "CUDA runtime error";
+    case ATTN_ENOMEM: return "workspace allocation failed";
+    case ATTN_ETIMEOUT: return "device-side wait timed out";
+    default: return "unknown error";
+  }
+}
+
+const char *attn_sink_last_error(void) { return t_last_error; }
+
+int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                  const attn_tensor *sinks, int32_t window, float scale, attn_tensor *out,
+                  attn_tensor *lse, void *stream) {
+  t_last_error[0] = '\0';
+  FwdArgs a;
+  int rc = prep_fwd(q, k, v, sinks, window, scale, out, lse, true, &a);
+  if (rc) return rc;
+  if (a.D != 64 && a.D != 128 && a.D != 256)
+    return fail(ATTN_EUNSUPPORTED, "head dim %d not supported (64, 128, 256)", a.D);
+  if (a.B == 0 || a.L == 0) return ATTN_OK;
+  if ((rc = status_ptr(&a.status))) return rc;
+  const cudaError_t e = launch_fwd_tc(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd launch");
+}
+
+int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                           const attn_tensor *sinks, int32_t window, float scale,
+                           attn_tensor *out, attn_tensor *lse, void *stream) {
+  t_last_error[0] = '\0';
+  FwdArgs a;
+  int rc = prep_fwd(q, k, v, sinks, window, scale, out, lse, false, &a);
+  if (rc) return rc;
+  if (a.D % 32 != 0 || a.D < 32 || a.D > 256)
+    return fail(ATTN_EUNSUPPORTED, "head dim %d not supported (multiple of 32, <= 256)", a.D);
+  if (a.B == 0 || a.L == 0) return ATTN_OK;
+  if ((rc = status_ptr(&a.status))) return rc;
+  const cudaError_t e = launch_fwd_cudacore(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd_cudacore launch");
+}
+
+int attn_sink_decode_chunked(const attn_tensor *q, const attn_tensor *kcache,
+                             const attn_tensor *vcache, const attn_tensor *seqlens,
+                             const attn_tensor *sinks, int32_t window, float scale,
+                             int32_t chunk, attn_tensor *out, void *stream) {
+  t_last_error[0] = '\0';
+  int rc;
+  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 3, false))) return rc;
+  if ((rc = check_tensor(kcache, "kcache", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(vcache, "vcache", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(seqlens, "seqlens", ATTN_DTYPE_I32, 1, false))) return rc;
+  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(out, "out", ATTN_DTYPE_BF16, 3, false))) return rc;
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t Smax = kcache->shape[1], Hkv = kcache->shape[2];
+  if (kcache->shape[0] != B || kcache->shape[3] != D) return fail(ATTN_EINVAL, "kcache shape does not match q");
+  for (int d = 0; d < 4; ++d)
+    if (vcache->shape[d] != kcache->shape[d]) return fail(ATTN_EINVAL, "vcache shape does not match kcache");
+  for (int d = 0; d < 3; ++d)
+    if (out->shape[d] != q->shape[d]) return fail(ATTN_EINVAL, "out shape does not match q");
+  if (seqlens->shape[0] != B) return fail(ATTN_EINVAL, "seqlens must have B entries");
+  if (sinks->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks must have Hq entries");
+  if ((B > 1 && seqlens->stride[0] != 1) || (Hq > 1 && sinks->stride[0] != 1))
+    return fail(ATTN_EINVAL, "seqlens and sinks must be contiguous");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
+  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
+  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
+  if (chunk < 0 || chunk % 64 != 0) return fail(ATTN_EINVAL, "chunk must be 0 or a positive multiple of 64");
+  if (D != 64 && D != 128 && D != 256) return fail(ATTN_EUNSUPPORTED, "head dim %lld not supported", (long long)D);
+  if (Hq / Hkv > (D == 256 ? 8 : 16)) return fail(ATTN_EUNSUPPORTED, "Hq/Hkv too large for this head dim");
+  if ((reinterpret_cast<uintptr_t>(q->data) % 4) || q->stride[0] % 2 || q->stride[1] % 2)
+    return fail(ATTN_EINVAL, "q rows must be 4-byte aligned");
+  if (B > (1 << 20) || Smax > (1LL << 30)) return fail(ATTN_EUNSUPPORTED, "B or Smax too large");
+  if (B == 0 || Hq == 0) return ATTN_OK;
+
+  DecodeArgs a;
+  a.q = q->data;
+  a.kc = kcache->data;
+  a.vc = vcache->data;
+  a.seqlens = static_cast<const int *>(seqlens->data);
+  a.sinks = static_cast<const float *>(sinks->data);
+  a.out = out->data;
+  a.B = static_cast<int>(B);
+  a.Smax = static_cast<int>(Smax);
+  a.Hq = static_cast<int>(Hq);
+  a.Hkv = static_cast<int>(Hkv);
+  a.D = static_cast<int>(D);
+  a.W = window;
+  a.scale = scale;
+  const int64_t vis = window < Smax ? window : Smax;
+  if (chunk == 0) {
+    // keep every sequence within 32 splits (the exact small-split combine)
+    int64_t c = ((vis + 31) / 32 + 63) / 64 * 64;
+    chunk = static_cast<int32_t>(c < 256 ? 256 : c);
+  }
+  a.chunk = chunk;
+  for (int d = 0; d < 2; ++d) {
+    a.q_s[d] = q->stride[d];
+    a.o_s[d] = out->stride[d];
+  }
+  for (int d = 0; d < 3; ++d) {
+    a.kc_s[d] = kcache->stride[d];
+    a.vc_s[d] = vcache->stride[d];
+  }
+  if ((rc = status_ptr(&a.status))) return rc;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  const size_t bytes = decode_workspace_bytes(a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void *ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, st);
+  if (e != cudaSuccess) return fail_cuda(e, "decode workspace allocation");
+  e = launch_decode(a, ws, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e != cudaSuccess) return fail_cuda(e, "attn_sink_decode launch");
+  if (ef != cudaSuccess) return fail_cuda(ef, "decode workspace release");
+  return ATTN_OK;
+}
+
+int attn_sink_decode(const attn_tensor *q, const attn_tensor *kcache, const attn_tensor *vcache,
+                     const attn_tensor *seqlens, const attn_tensor *sinks, int32_t window,
+                     float scale, attn_tensor *out, void *stream) {
+  return attn_sink_decode_chunked(q, kcache, vcache, seqlens, sinks, window, scale, 0, out, stream);
+}
+
+int attn_sink_get_status(void *stream) {
+  t_last_error[0] = '\0';
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "cudaStreamSynchronize");
+  int *dptr;
+  int rc = status_ptr(&dptr);
+  if (rc) return rc;
+  int h[2] = {0, 0};
+  e = cudaMemcpy(h, dptr, sizeof h, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e, "status read");
+  if (h[0] != 0) {
+    const int zero[2] = {0, 0};
+    e = cudaMemcpy(dptr, zero, sizeof zero, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return fail_cuda(e, "status reset");
+    return fail(h[0], "device wait timed out at location %d", h[1]);
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,597 @@
+// decode.cu -- single-token split-KV decode with a learned per-head sink.
+//
+// Three kernels on one stream, no host synchronisation:
+//   plan     reads seqlens on the device; splits each sequence's visible key
+//            range [max(0, n-W), n) into chunks of `chunk` keys and lays the
+//            splits out contiguously (split_base[b] = exclusive prefix sum).
+//   split    persistent: one work item = (split, kv head).  A TMA producer
+//            warp streams 64-key K/V tiles of that head into a ring of stages;
+//            four consumer warps each take 16 keys of every tile and run
+//            S^T = K q^T and O^T += V^T P^T on the warp-level tensor cores
+//            (the Hq/Hkv grouped query heads are the N = 8 dimension), with an
+//            online softmax per head and NO sink.  At the end of an item the
+//            four warps' (max, sum, O) are merged and one normalised partial
+//            (O_s, LSE_s) per query head is written.
+//   combine  one warp per (sequence, query head): merges exactly the splits
+//            that exist, in split order, and adds the sink once.
+// Split-KV decode and the LSE combine: page
+// "flashmla-optimization/docs/PATCH_STACK.md", section 3 ("exact small-split
+// combine": with <= 32 real splits only the valid LSE lanes are reduced and no
+// masked work is built for splits that do not exist; the accumulation order of
+// the real splits is kept).  The sink term is the learned sink of page
+// "cf-1.com/news/6055759".
+//
+// Decode moves ~512 bytes of K/V per key per kv head for 8 x 128 x 4 flops, so
+// it is bound by HBM bandwidth; the warp-level MMA keeps the arithmetic far
+// below that bound without tying up registers in fp32 FMA loops.
+#include <math.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace attnsink {
+namespace {
+
+constexpr int kTK = 64;               // keys per tile
+constexpr int kConsumerWarps = 4;     // each owns 16 keys of every tile
+constexpr int kProducerWarp = 4;
+constexpr int kThreads = 5 * 32;
+constexpr uint32_t kBarMerge = 1;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+enum : int { kWhereFull = 201, kWhereEmpty = 202 };
+
+// Workspace layout (each section 256-byte aligned).
+struct WsLayout {
+  size_t off_nsplit, off_base, off_ctrl, off_lse, off_o, total;
+  int max_splits;  // upper bound on the total number of splits
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(const DecodeArgs &a) {
+  WsLayout w;
+  const int per_seq = decode_max_splits_per_seq(a);
+  w.max_splits = a.B * per_seq;
+  size_t off = 0;
+  w.off_nsplit = off;
+  off = align256(off + sizeof(int) * a.B);
+  w.off_base = off;
+  off = align256(off + sizeof(int) * a.B);
+  w.off_ctrl = off;                                   // [0] total splits, [1] work counter
+  off = align256(off + sizeof(int) * 4);
+  w.off_lse = off;
+  off = align256(off + sizeof(float) * static_cast<size_t>(w.max_splits) * a.Hq);
+  w.off_o = off;
+  off = align256(off + sizeof(float) * static_cast<size_t>(w.max_splits) * a.Hq * a.D);
+  w.total = off;
+  return w;
+}
+
+// ------------------------------------------------------------------- plan
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const int *seqlens, int B, int Smax,
+                                                           int W, int chunk, int *nsplit,
+                                                           int *base, int *ctrl) {
+  __shared__ int warp_sums[32];
+  const int t = threadIdx.x;
+  const int per = (B + blockDim.x - 1) / blockDim.x;  // contiguous segment per thread
+  const int b0 = t * per;
+  int local = 0;
+  for (int b = b0; b < min(B, b0 + per); ++b) {
+    const int n = min(max(seqlens[b], 0), Smax);
+    const int len = n - max(0, n - W);
+    const int ns = (len + chunk - 1) / chunk;
+    nsplit[b] = ns;
+    local += ns;
+  }
+  // block-wide exclusive scan of the per-thread sums
+  const int lane = t & 31, wid = t >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    const int nw = blockDim.x >> 5;
+    int v = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < nw) warp_sums[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = incl - local + (wid > 0 ? warp_sums[wid - 1] : 0);
+  for (int b = b0; b < min(B, b0 + per); ++b) {
+    base[b] = run;
+    run += nsplit[b];
+  }
+  if (t == blockDim.x - 1) {
+    ctrl[0] = run;  // total splits
+    ctrl[1] = 0;    // work counter for the split kernel
+  }
+}
+
+// ------------------------------------------------------------------ split
+struct SplitParams {
+  const __nv_bfloat16 *q;
+  int64_t q_sb, q_sh;
+  const int *seqlens;
+  const int *nsplit, *base, *ctrl;
+  int *work_counter;
+  float *lse_part, *o_part;
+  int B, Smax, Hq, Hkv, G, W, chunk;
+  float scale_log2;
+  int *status;
+};
+
+struct StageInfo {
+  int b, hk, split, key0, nvalid, flags;  // flags: 1 first tile, 2 last tile, 4 end of work
+  int pad[2];
+};
+
+template <int D, int NT>
+struct DCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kTK * D * 2;          // one K (or V) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
+  static constexpr int kStages = (196608 / kStageBytes) > 12 ? 12 : (196608 / kStageBytes);
+  static constexpr int kMergeBytes = kConsumerWarps * NT * 8 * D * 4;
+  static constexpr int kInfoOffset = kStages * kStageBytes + kMergeBytes;
+  static constexpr int kSmemBytes = kInfoOffset + 1024 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const WaitCtx &ctx,
+                                          int where) {
+  const bool r = mbar_wait(bar, parity, ctx, where);
+  return __all_sync(0xffffffffu, r);
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const SplitParams p) {
+  using C = DCfg<D, NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  float *merge = reinterpret_cast<float *>(smem + C::kStages * C::kStageBytes);
+  StageInfo *info = reinterpret_cast<StageInfo *>(smem + C::kInfoOffset);
+  uint64_t *full = reinterpret_cast<uint64_t *>(info + C::kStages);
+  uint64_t *empty = full + C::kStages;
+  float *merge_m = reinterpret_cast<float *>(empty + C::kStages);   // [4][NT*8]
+  float *merge_l = merge_m + kConsumerWarps * NT * 8;               // [4][NT*8]
+  int *abort_flag = reinterpret_cast<int *>(merge_l + kConsumerWarps * NT * 8);
+  const WaitCtx ctx{abort_flag, p.status};
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kProducerWarp) {
+    // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int total_items = p.ctrl[0] * p.Hkv;
+      int slot = 0;
+      bool ok = true;
+      auto acquire = [&]() -> int {
+        const int s = slot % C::kStages;
+        const uint32_t use = static_cast<uint32_t>(slot / C::kStages);
+        if (slot >= C::kStages && !mbar_wait(&empty[s], (use & 1u) ^ 1u, ctx, kWhereEmpty))
+          ok = false;
+        ++slot;
+        return s;
+      };
+      while (ok) {
+        const int w = atomicAdd(p.work_counter, 1);
+        if (w >= total_items) break;
+        const int g = w / p.Hkv, hk = w - g * p.Hkv;
+        int lo = 0, hi = p.B - 1;  // last b with base[b] <= g
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (p.base[mid] <= g) lo = mid; else hi = mid - 1;
+        }
+        const int b = lo;
+        const int split = g - p.base[b];
+        const int n = min(max(p.seqlens[b], 0), p.Smax);
+        const int ks = max(0, n - p.W) + split * p.chunk;
+        const int ke = min(n, ks + p.chunk);
+        const int nt = (ke - ks + kTK - 1) / kTK;
+        for (int t = 0; ok && t < nt; ++t) {
+          const int s = acquire();
+          if (!ok) break;
+          StageInfo &si = info[s];
+          si.b = b;
+          si.hk = hk;
+          si.split = split;
+          si.key0 = ks + t * kTK;
+          si.nvalid = min(kTK, ke - si.key0);
+          si.flags = (t == 0 ? 1 : 0) | (t == nt - 1 ? 2 : 0);
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          uint8_t *dst = smem + s * C::kStageBytes;
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_4d(dst + c * kTK * 128, &tmK, &full[s], c * 64, hk, si.key0, b);
+            tma_load_4d(dst + C::kTileBytes + c * kTK * 128, &tmV, &full[s], c * 64, hk, si.key0, b);
+          }
+        }
+      }
+      if (ok) {
+        const int s = acquire();
+        if (ok) {
+          info[s].flags = 4;
+          mbar_arrive(&full[s]);
+        }
+      }
+    }
+    __syncwarp();
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int g8 = lane >> 2;       // mma "group" (row within an 8-row block)
+  const int tig = lane & 3;       // thread in group
+  const float sl2 = p.scale_log2;
+  uint32_t qf[D / 16][NT][2];     // B fragments of q^T, per k-step and head tile
+  float o[D / 16][NT][4];         // O^T accumulators: [d tile][head tile][frag]
+  float m_run[NT][2], l_run[NT][2];
+  int slot = 0;
+  while (true) {
+    const int s = slot % C::kStages;
+    if (!warp_wait(&full[s], static_cast<uint32_t>(slot / C::kStages) & 1u, ctx, kWhereFull)) break;
+    ++slot;
+    const StageInfo si = info[s];
+    if (si.flags & 4) break;
+    const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
+    const uint32_t vbase = kbase + C::kTileBytes;
+    if (si.flags & 1) {
+      // first tile of a work item: load this kv head's grouped queries
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hl = nt * 8 + g8;
+          uint32_t x0 = 0, x1 = 0;
+          if (hl < p.G) {
+            const __nv_bfloat16 *qr = p.q + si.b * p.q_sb + (si.hk * p.G + hl) * p.q_sh + kk * 16 + 2 * tig;
+            x0 = *reinterpret_cast<const uint32_t *>(qr);
+            x1 = *reinterpret_cast<const uint32_t *>(qr + 8);
+          }
+          qf[kk][nt][0] = x0;
+          qf[kk][nt][1] = x1;
+        }
+#pragma unroll
+      for (int dm = 0; dm < D / 16; ++dm)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int f = 0; f < 4; ++f) o[dm][nt][f] = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        m_run[nt][0] = m_run[nt][1] = -INFINITY;
+        l_run[nt][0] = l_run[nt][1] = 0.f;
+      }
+    }
+    const int key_w = warp * 16;  // this warp's 16 keys within the tile
+    // Keys past the end of the split are masked; where they are past the end
+    // of the sequence their cache rows may hold anything (NaN included), so
+    // their V rows are zeroed in shared memory before P.V reads them.
+    if (si.nvalid < key_w + 16) {
+      const int kidx = key_w + (lane & 15);
+      if (kidx >= si.nvalid) {
+        for (int c = 0; c < C::kChunks; ++c) {
+          uint8_t *row = smem + s * C::kStageBytes + C::kTileBytes + c * kTK * 128 + kidx * 128;
+          const int half = lane >> 4;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4 *>(row + (half * 4 + u) * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      __syncwarp();
+    }
+    // ---- S^T[16 keys x 8*NT heads] = K_w q^T ----
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int f = 0; f < 4; ++f) sacc[nt][f] = 0.f;
+    {
+      const int krow = key_w + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int unit = 2 * (kk & 3) + (lane >> 4);
+        const uint32_t addr = kbase + (kk >> 2) * (kTK * 128) + krow * 128 + ((unit ^ (krow & 7)) << 4);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+      }
+    }
+    // ---- online softmax per head (no sink here) ----
+    const bool v0 = key_w + g8 < si.nvalid, v1 = key_w + g8 + 8 < si.nvalid;
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float x[4];
+      x[0] = v0 ? sacc[nt][0] * sl2 : -INFINITY;  // key g,   head 2tig
+      x[1] = v0 ? sacc[nt][1] * sl2 : -INFINITY;  // key g,   head 2tig+1
+      x[2] = v1 ? sacc[nt][2] * sl2 : -INFINITY;  // key g+8, head 2tig
+      x[3] = v1 ? sacc[nt][3] * sl2 : -INFINITY;  // key g+8, head 2tig+1
+      float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float n0 = fmaxf(m_run[nt][0], mx0), n1 = fmaxf(m_run[nt][1], mx1);
+      const float a0 = (n0 == -INFINITY) ? 1.f : ex2_approx(m_run[nt][0] - n0);
+      const float a1 = (n1 == -INFINITY) ? 1.f : ex2_approx(m_run[nt][1] - n1);
+      m_run[nt][0] = n0;
+      m_run[nt][1] = n1;
+      const float u0 = (n0 == -INFINITY) ? 0.f : n0, u1 = (n1 == -INFINITY) ? 0.f : n1;
+      const float p0 = ex2_approx(x[0] - u0), p1 = ex2_approx(x[1] - u1);
+      const float p2 = ex2_approx(x[2] - u0), p3 = ex2_approx(x[3] - u1);
+      l_run[nt][0] = l_run[nt][0] * a0 + p0 + p2;
+      l_run[nt][1] = l_run[nt][1] * a1 + p1 + p3;
+      if (a0 != 1.f || a1 != 1.f) {
+#pragma unroll
+        for (int dm = 0; dm < D / 16; ++dm) {
+          o[dm][nt][0] *= a0;
+          o[dm][nt][1] *= a1;
+          o[dm][nt][2] *= a0;
+          o[dm][nt][3] *= a1;
+        }
+      }
+      // P^T fragments (key rows, head columns) -> transposed into the
+      // B-operand layout of O^T += V^T P^T.
+      pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+      pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+    }
+    // ---- O^T[D x 8*NT] += V_w^T P^T ----
+    {
+      const int vrow = key_w + (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+      for (int dm = 0; dm < D / 16; ++dm) {
+        const int unit = 2 * (dm & 3) + ((lane >> 3) & 1);
+        const uint32_t addr = vbase + (dm >> 2) * (kTK * 128) + vrow * 128 + ((unit ^ (vrow & 7)) << 4);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      }
+    }
+    // release the stage (generic-proxy writes above are ordered before the
+    // next TMA write into it)
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+
+    if (si.flags & 2) {
+      // ---- merge the four warps' partial states and write (O_s, LSE_s) ----
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float l = l_run[nt][e];
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+          l_run[nt][e] = l;
+        }
+      named_barrier_sync(kBarMerge, kConsumerWarps * 32);  // previous merge fully read
+      if (g8 == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            merge_m[warp * NT * 8 + nt * 8 + 2 * tig + e] = m_run[nt][e];
+            merge_l[warp * NT * 8 + nt * 8 + 2 * tig + e] = l_run[nt][e];
+          }
+      }
+      float *mw = merge + warp * (NT * 8 * D);  // [head][d]
+#pragma unroll
+      for (int dm = 0; dm < D / 16; ++dm)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hh = nt * 8 + 2 * tig;
+          mw[hh * D + dm * 16 + g8] = o[dm][nt][0];
+          mw[(hh + 1) * D + dm * 16 + g8] = o[dm][nt][1];
+          mw[hh * D + dm * 16 + g8 + 8] = o[dm][nt][2];
+          mw[(hh + 1) * D + dm * 16 + g8 + 8] = o[dm][nt][3];
+        }
+      named_barrier_sync(kBarMerge, kConsumerWarps * 32);
+      const int tid = threadIdx.x;  // 0..127
+      const int gsplit = p.base[si.b] + si.split;
+      for (int e = tid; e < p.G * D; e += kConsumerWarps * 32) {
+        const int hh = e / D, d = e - hh * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w * NT * 8 + hh]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw_ = merge_m[w * NT * 8 + hh];
+          const float f = (mw_ == -INFINITY) ? 0.f : ex2_approx(mw_ - M);
+          num += f * merge[w * (NT * 8 * D) + hh * D + d];
+          den += f * merge_l[w * NT * 8 + hh];
+        }
+        const int hq = si.hk * p.G + hh;
+        const size_t row = static_cast<size_t>(gsplit) * p.Hq + hq;
+        p.o_part[row * D + d] = num / den;
+        if (d == 0) p.lse_part[row] = (M + log2f(den)) * kLn2;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- combine
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const int *nsplit, const int *base,
+                                                             const float *lse_part,
+                                                             const float *o_part,
+                                                             const float *sinks,
+                                                             __nv_bfloat16 *out, int64_t o_sb,
+                                                             int64_t o_sh, int B, int Hq) {
+  constexpr int DPL = D / 32;
+  const int wg = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wg >= B * Hq) return;
+  const int b = wg / Hq, hq = wg - b * Hq;
+  const int ns = nsplit[b];
+  const int sb = base[b];
+  const float sink = sinks[hq];
+  float acc[DPL];
+#pragma unroll
+  for (int t = 0; t < DPL; ++t) acc[t] = 0.f;
+  float M = sink, den;
+  if (ns <= 32) {
+    // Exact small-split path: only the lanes of splits that exist hold an LSE.
+    const float ls = lane < ns ? lse_part[static_cast<size_t>(sb + lane) * Hq + hq] : -INFINITY;
+    float mx = ls;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    M = fmaxf(M, mx);
+    const float w = lane < ns ? __expf(ls - M) : 0.f;
+    float sw = w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, off);
+    den = sw + ((sink == -INFINITY) ? 0.f : __expf(sink - M));
+    for (int s = 0; s < ns; ++s) {  // split order 0, 1, 2, ...
+      const float ws = __shfl_sync(0xffffffffu, w, s);
+      const float *op = o_part + (static_cast<size_t>(sb + s) * Hq + hq) * D;
+#pragma unroll
+      for (int t = 0; t < DPL; ++t) acc[t] = fmaf(ws, op[lane + 32 * t], acc[t]);
+    }
+  } else {
+    // General path for more than 32 splits (same arithmetic, chunked).
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      const float ls = s0 + lane < ns ? lse_part[static_cast<size_t>(sb + s0 + lane) * Hq + hq] : -INFINITY;
+      float mx = ls;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      M = fmaxf(M, mx);
+    }
+    float sw = 0.f;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      const float ls = s0 + lane < ns ? lse_part[static_cast<size_t>(sb + s0 + lane) * Hq + hq] : -INFINITY;
+      const float w = s0 + lane < ns ? __expf(ls - M) : 0.f;
+      float t_ = w;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) t_ += __shfl_xor_sync(0xffffffffu, t_, off);
+      sw += t_;
+      const int cnt = min(32, ns - s0);
+      for (int s = 0; s < cnt; ++s) {
+        const float ws = __shfl_sync(0xffffffffu, w, s);
+        const float *op = o_part + (static_cast<size_t>(sb + s0 + s) * Hq + hq) * D;
+#pragma unroll
+        for (int t = 0; t < DPL; ++t) acc[t] = fmaf(ws, op[lane + 32 * t], acc[t]);
+      }
+    }
+    den = sw + ((sink == -INFINITY) ? 0.f : __expf(sink - M));
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  __nv_bfloat16 *orow = out + b * o_sb + hq * o_sh;
+#pragma unroll
+  for (int t = 0; t < DPL; ++t) orow[lane + 32 * t] = __float2bfloat16_rn(acc[t] * inv);
+}
+
+template <int D, int NT>
+cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cudaStream_t stream) {
+  using C = DCfg<D, NT>;
+  alignas(64) CUtensorMap mk, mv;
+  cudaError_t e;
+  if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, kTK)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, kTK)) != cudaSuccess) return e;
+  SplitParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(a.q);
+  p.q_sb = a.q_s[0];
+  p.q_sh = a.q_s[1];
+  p.seqlens = a.seqlens;
+  p.nsplit = reinterpret_cast<const int *>(ws + w.off_nsplit);
+  p.base = reinterpret_cast<const int *>(ws + w.off_base);
+  p.ctrl = reinterpret_cast<const int *>(ws + w.off_ctrl);
+  p.work_counter = reinterpret_cast<int *>(ws + w.off_ctrl) + 1;
+  p.lse_part = reinterpret_cast<float *>(ws + w.off_lse);
+  p.o_part = reinterpret_cast<float *>(ws + w.off_o);
+  p.B = a.B;
+  p.Smax = a.Smax;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.W = a.W;
+  p.chunk = a.chunk;
+  p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
+  p.status = a.status;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long items = static_cast<long long>(w.max_splits) * a.Hkv;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  if (grid <= 0) return cudaSuccess;
+  auto kern = decode_split_kernel<D, NT>;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes)) !=
+      cudaSuccess)
+    return e;
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mk, mv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_combine(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(a.B) * a.Hq;
+  const int blocks = static_cast<int>((warps * 32 + 127) / 128);
+  decode_combine_kernel<D><<<blocks, 128, 0, stream>>>(
+      reinterpret_cast<const int *>(ws + w.off_nsplit), reinterpret_cast<const int *>(ws + w.off_base),
+      reinterpret_cast<const float *>(ws + w.off_lse), reinterpret_cast<const float *>(ws + w.off_o),
+      a.sinks, static_cast<__nv_bfloat16 *>(a.out), a.o_s[0], a.o_s[1], a.B, a.Hq);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_max_splits_per_seq(const DecodeArgs &a) {
+  const long long vis = a.W < a.Smax ? a.W : a.Smax;
+  return static_cast<int>((vis + a.chunk - 1) / a.chunk);
+}
+
+size_t decode_workspace_bytes(const DecodeArgs &a) { return ws_layout(a).total; }
+
+cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t stream) {
+  const WsLayout w = ws_layout(a);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  decode_plan_kernel<<<1, 1024, 0, stream>>>(a.seqlens, a.B, a.Smax, a.W, a.chunk,
+                                             reinterpret_cast<int *>(ws + w.off_nsplit),
+                                             reinterpret_cast<int *>(ws + w.off_base),
+                                             reinterpret_cast<int *>(ws + w.off_ctrl));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int G = a.Hq / a.Hkv;
+  switch (a.D) {
+    case 64: e = G <= 8 ? launch_split<64, 1>(a, w, ws, stream) : launch_split<64, 2>(a, w, ws, stream); break;
+    case 128: e = G <= 8 ? launch_split<128, 1>(a, w, ws, stream) : launch_split<128, 2>(a, w, ws, stream); break;
+    case 256: e = G <= 8 ? launch_split<256, 1>(a, w, ws, stream) : cudaErrorInvalidValue; break;
+    default: e = cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  switch (a.D) {
+    case 64: return launch_combine<64>(a, w, ws, stream);
+    case 128: return launch_combine<128>(a, w, ws, stream);
+    case 256: return launch_combine<256>(a, w, ws, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace attnsink

@@ -1,0 +1,55 @@
+// kernels.h -- host-side interface between the C ABI (api.cu) and the kernel
+// launchers.  Arguments arrive here already validated; strides are in
+// elements and the innermost dimension of every tensor is contiguous.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace attnsink {
+
+// Prefill forward: q/out [B,L,Hq,D], k/v [B,L,Hkv,D] (bf16), sinks [Hq] f32,
+// lse [B,Hq,L] f32 or null.
+struct FwdArgs {
+  const void *q, *k, *v;
+  const float *sinks;
+  void *out;
+  float *lse;
+  int B, L, Hq, Hkv, D, W;
+  float scale;
+  int64_t q_s[3], k_s[3], v_s[3], o_s[3];  // strides of dims 0..2
+  int64_t lse_s[2];                        // strides of dims 0..1
+  int *status;                             // device status word (2 ints)
+};
+
+// Decode: q/out [B,Hq,D], caches [B,Smax,Hkv,D] (bf16), seqlens [B] int32
+// (device), sinks [Hq] f32.
+struct DecodeArgs {
+  const void *q, *kc, *vc;
+  const int *seqlens;
+  const float *sinks;
+  void *out;
+  int B, Smax, Hq, Hkv, D, W;
+  float scale;
+  int chunk;                               // keys per split (multiple of 64)
+  int64_t q_s[2], kc_s[3], vc_s[3], o_s[2];
+  int *status;
+};
+
+// Bytes of stream-ordered workspace one decode call needs (256-byte aligned
+// sections: plan, partial LSEs, partial outputs).
+size_t decode_workspace_bytes(const DecodeArgs &a);
+// Upper bound on the number of splits of one sequence for these arguments.
+int decode_max_splits_per_seq(const DecodeArgs &a);
+
+cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream);
+cudaError_t launch_fwd_cudacore(const FwdArgs &a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t stream);
+
+// Builds a 4-D TMA descriptor for a [d3,d2,d1,d0] bf16 tensor (d0 innermost,
+// contiguous) with 128-byte swizzle and a box of {64, 1, box_rows, 1}, i.e.
+// box_rows consecutive positions of one head and 64 of its channels.
+// Returns cudaErrorInvalidValue if the driver rejects the description.
+cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
+                          int64_t d0, const int64_t strides_el[3], int box_rows);
+
+}  // namespace attnsink
