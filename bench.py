@@ -96,7 +96,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.idx), "-lms", "100"],
+                 "-i", str(self.idx), "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -325,7 +325,7 @@ def cpu_baseline(budget_s: float = 10.0):
     t0 = time.perf_counter()
     run()
     dt = time.perf_counter() - t0
-    n_rows = int(max(256, min(200000, 256 * budget_s / max(dt, 1e-6))))
+    n_rows = int(max(256, min(4000000, 256 * budget_s / max(dt, 1e-6))))
     run, flops = _oracle_sample(n_rows, seed=1)
     t0 = time.perf_counter()
     run()
@@ -376,7 +376,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
