@@ -1,0 +1,64 @@
+"""Runs a few launches of one operation on a chosen workload, for profiler
+captures (Nsight Compute) of a single kernel on a bounded device footprint.
+
+  python -m sliding_window_learned_b200.ncu_driver --op fwd --workload prefill --launches 3
+  python -m sliding_window_learned_b200.ncu_driver --op decode --workload decode-small --launches 3
+
+It prints no timings (numbers taken under a profiler are not measurements);
+it exits non-zero if the device reports an error.
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+import torch
+
+from . import abi, build, inputs
+
+WORKLOADS = {
+    "tiny": inputs.TINY,
+    "prefill": inputs.PREFILL,
+    "long-causal": inputs.LONG_CAUSAL,
+    "stress": inputs.STRESS,
+    "decode": inputs.DECODE,
+    # same length distribution as the decode workload, 8 sequences (~1 GB of cache)
+    "decode-small": inputs.Decode("decode-small B8 Hq32 Hkv4 D128 n~U[4096,131072]", 8, 32, 4,
+                                  128, 131072, 4096, 131072, 131072),
+}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", choices=["fwd", "decode"], required=True)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
+    ap.add_argument("--launches", type=int, default=3)
+    a = ap.parse_args(argv)
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = WORKLOADS[a.workload]
+    if a.op == "fwd":
+        if not isinstance(cfg, inputs.Prefill):
+            raise SystemExit("fwd needs a prefill workload")
+        x = inputs.make_prefill(cfg, seed=0, device=dev)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty(cfg.B, cfg.Hq, cfg.L, dtype=torch.float32, device=dev)
+        for _ in range(a.launches):
+            abi.attn_sink_fwd(x["q"], x["k"], x["v"], x["sinks"], cfg.W, cfg.scale, out, lse)
+    else:
+        if not isinstance(cfg, inputs.Decode):
+            raise SystemExit("decode needs a decode workload")
+        y = inputs.make_decode(cfg, seed=0, device=dev)
+        out = torch.empty_like(y["q"])
+        for _ in range(a.launches):
+            abi.attn_sink_decode(y["q"], y["kcache"], y["vcache"], y["seqlens"], y["sinks"],
+                                 cfg.W, cfg.scale, out)
+    torch.cuda.synchronize()
+    rc = abi.attn_sink_get_status()
+    print("ok" if rc == 0 else f"device status {rc}")
+    return 0 if rc == 0 else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main())
