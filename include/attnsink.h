@@ -138,6 +138,35 @@ int attn_sink_decode_chunked(const attn_tensor *q, const attn_tensor *kcache,
                              int32_t chunk, attn_tensor *out, void *stream);
 
 /*
+ * attn_sink_decode without any allocation (the pages have no counterpart to
+ * this entry point; it is a deployment convenience).  Same arguments, result
+ * and kernels as attn_sink_decode, but the split table and the partial
+ * (O_s, LSE_s) live in a fixed 48 MiB array of device memory inside the
+ * library instead of a stream-ordered allocation.  It is meant for callers
+ * that may not allocate device memory while they decode: engines that
+ * reserve nearly all of HBM for their KV cache up front and forbid library
+ * allocations, or runtimes whose own allocator owns every device byte.
+ *
+ *  - Nothing is allocated or freed: no cudaMalloc/cudaFree of any kind.
+ *  - The array is part of the library's device image: every GPU on which this
+ *    entry point is used holds the 48 MiB until the process exits.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Workloads whose workspace bound exceeds 48 MiB are rejected with
+ *    ATTN_EUNSUPPORTED and a message giving both sizes.  The bound is
+ *    B * ceil(min(Smax, window) / chunk) * Hq * (D + 1) * 4 bytes, with the
+ *    library's default chunk (every sequence <= 32 splits), plus ~1 KB.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (each call rewrites everything it reads).  Calls whose kernels
+ *    overlap on the GPU -- concurrent streams, or threads driving the same
+ *    device -- race on it; serialise them (e.g. one stream).
+ */
+int attn_sink_decode_noalloc(const attn_tensor *q, const attn_tensor *kcache,
+                             const attn_tensor *vcache, const attn_tensor *seqlens,
+                             const attn_tensor *sinks, int32_t window, float scale,
+                             attn_tensor *out, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, ATTN_ETIMEOUT (a bounded wait ran out), or
  * ATTN_ECUDA if the synchronisation itself failed.

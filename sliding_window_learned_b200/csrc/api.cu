@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/attnsink.h"
+#include "api_internal.h"
 #include "kernels.h"
 
 namespace attnsink {
@@ -21,8 +22,10 @@ namespace attnsink {
 __device__ int g_status[2];
 
 namespace {
-
 thread_local char t_last_error[256] = "";
+}  // namespace
+
+void clear_error() { t_last_error[0] = '\0'; }
 
 int fail(int code, const char *fmt, ...) {
   va_list ap;
@@ -37,11 +40,14 @@ int fail_cuda(cudaError_t e, const char *what) {
               cudaGetErrorString(e));
 }
 
+namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int *g_status_ptr[kMaxDevices];
 cudaMemPool_t g_pool[kMaxDevices];
 bool g_pool_ready[kMaxDevices];
+
+}  // namespace
 
 int current_device(int *dev) {
   const cudaError_t e = cudaGetDevice(dev);
@@ -64,6 +70,8 @@ int status_ptr(int **out) {
   *out = g_status_ptr[dev];
   return ATTN_OK;
 }
+
+namespace {
 
 // A private stream-ordered pool per device that keeps freed blocks cached, so
 // repeated decode calls reuse their workspace without new mappings.
@@ -214,6 +222,75 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Validates the decode arguments and fills `out_args`; `*empty` is set when
+// there is nothing to compute (B == 0 or Hq == 0).
+int prep_decode(const attn_tensor *q, const attn_tensor *kcache, const attn_tensor *vcache,
+                const attn_tensor *seqlens, const attn_tensor *sinks, int32_t window, float scale,
+                int32_t chunk, attn_tensor *out, DecodeArgs *out_args, bool *empty) {
+  int rc;
+  *empty = false;
+  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 3, false))) return rc;
+  if ((rc = check_tensor(kcache, "kcache", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(vcache, "vcache", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(seqlens, "seqlens", ATTN_DTYPE_I32, 1, false))) return rc;
+  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(out, "out", ATTN_DTYPE_BF16, 3, false))) return rc;
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t Smax = kcache->shape[1], Hkv = kcache->shape[2];
+  if (kcache->shape[0] != B || kcache->shape[3] != D) return fail(ATTN_EINVAL, "kcache shape does not match q");
+  for (int d = 0; d < 4; ++d)
+    if (vcache->shape[d] != kcache->shape[d]) return fail(ATTN_EINVAL, "vcache shape does not match kcache");
+  for (int d = 0; d < 3; ++d)
+    if (out->shape[d] != q->shape[d]) return fail(ATTN_EINVAL, "out shape does not match q");
+  if (seqlens->shape[0] != B) return fail(ATTN_EINVAL, "seqlens must have B entries");
+  if (sinks->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks must have Hq entries");
+  if ((B > 1 && seqlens->stride[0] != 1) || (Hq > 1 && sinks->stride[0] != 1))
+    return fail(ATTN_EINVAL, "seqlens and sinks must be contiguous");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
+  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
+  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
+  if (chunk < 0 || chunk % 64 != 0) return fail(ATTN_EINVAL, "chunk must be 0 or a positive multiple of 64");
+  if (D != 64 && D != 128 && D != 256) return fail(ATTN_EUNSUPPORTED, "head dim %lld not supported", (long long)D);
+  if (Hq / Hkv > (D == 256 ? 8 : 16)) return fail(ATTN_EUNSUPPORTED, "Hq/Hkv too large for this head dim");
+  if ((reinterpret_cast<uintptr_t>(q->data) % 4) || q->stride[0] % 2 || q->stride[1] % 2)
+    return fail(ATTN_EINVAL, "q rows must be 4-byte aligned");
+  if (B > (1 << 20) || Smax > (1LL << 30)) return fail(ATTN_EUNSUPPORTED, "B or Smax too large");
+  if (B == 0 || Hq == 0) {
+    *empty = true;
+    return ATTN_OK;
+  }
+  DecodeArgs &a = *out_args;
+  a.q = q->data;
+  a.kc = kcache->data;
+  a.vc = vcache->data;
+  a.seqlens = static_cast<const int *>(seqlens->data);
+  a.sinks = static_cast<const float *>(sinks->data);
+  a.out = out->data;
+  a.B = static_cast<int>(B);
+  a.Smax = static_cast<int>(Smax);
+  a.Hq = static_cast<int>(Hq);
+  a.Hkv = static_cast<int>(Hkv);
+  a.D = static_cast<int>(D);
+  a.W = window;
+  a.scale = scale;
+  const int64_t vis = window < Smax ? window : Smax;
+  if (chunk == 0) {
+    // keep every sequence within 32 splits (the exact small-split combine)
+    int64_t c = ((vis + 31) / 32 + 63) / 64 * 64;
+    chunk = static_cast<int32_t>(c < 256 ? 256 : c);
+  }
+  a.chunk = chunk;
+  for (int d = 0; d < 2; ++d) {
+    a.q_s[d] = q->stride[d];
+    a.o_s[d] = out->stride[d];
+  }
+  for (int d = 0; d < 3; ++d) {
+    a.kc_s[d] = kcache->stride[d];
+    a.vc_s[d] = vcache->stride[d];
+  }
+  return ATTN_OK;
+}
+
 }  // namespace attnsink
 
 using namespace attnsink;
@@ -269,64 +346,10 @@ int attn_sink_decode_chunked(const attn_tensor *q, const attn_tensor *kcache,
                              const attn_tensor *sinks, int32_t window, float scale,
                              int32_t chunk, attn_tensor *out, void *stream) {
   t_last_error[0] = '\0';
-  int rc;
-  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 3, false))) return rc;
-  if ((rc = check_tensor(kcache, "kcache", ATTN_DTYPE_BF16, 4, true))) return rc;
-  if ((rc = check_tensor(vcache, "vcache", ATTN_DTYPE_BF16, 4, true))) return rc;
-  if ((rc = check_tensor(seqlens, "seqlens", ATTN_DTYPE_I32, 1, false))) return rc;
-  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
-  if ((rc = check_tensor(out, "out", ATTN_DTYPE_BF16, 3, false))) return rc;
-  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
-  const int64_t Smax = kcache->shape[1], Hkv = kcache->shape[2];
-  if (kcache->shape[0] != B || kcache->shape[3] != D) return fail(ATTN_EINVAL, "kcache shape does not match q");
-  for (int d = 0; d < 4; ++d)
-    if (vcache->shape[d] != kcache->shape[d]) return fail(ATTN_EINVAL, "vcache shape does not match kcache");
-  for (int d = 0; d < 3; ++d)
-    if (out->shape[d] != q->shape[d]) return fail(ATTN_EINVAL, "out shape does not match q");
-  if (seqlens->shape[0] != B) return fail(ATTN_EINVAL, "seqlens must have B entries");
-  if (sinks->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks must have Hq entries");
-  if ((B > 1 && seqlens->stride[0] != 1) || (Hq > 1 && sinks->stride[0] != 1))
-    return fail(ATTN_EINVAL, "seqlens and sinks must be contiguous");
-  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
-  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
-  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
-  if (chunk < 0 || chunk % 64 != 0) return fail(ATTN_EINVAL, "chunk must be 0 or a positive multiple of 64");
-  if (D != 64 && D != 128 && D != 256) return fail(ATTN_EUNSUPPORTED, "head dim %lld not supported", (long long)D);
-  if (Hq / Hkv > (D == 256 ? 8 : 16)) return fail(ATTN_EUNSUPPORTED, "Hq/Hkv too large for this head dim");
-  if ((reinterpret_cast<uintptr_t>(q->data) % 4) || q->stride[0] % 2 || q->stride[1] % 2)
-    return fail(ATTN_EINVAL, "q rows must be 4-byte aligned");
-  if (B > (1 << 20) || Smax > (1LL << 30)) return fail(ATTN_EUNSUPPORTED, "B or Smax too large");
-  if (B == 0 || Hq == 0) return ATTN_OK;
-
   DecodeArgs a;
-  a.q = q->data;
-  a.kc = kcache->data;
-  a.vc = vcache->data;
-  a.seqlens = static_cast<const int *>(seqlens->data);
-  a.sinks = static_cast<const float *>(sinks->data);
-  a.out = out->data;
-  a.B = static_cast<int>(B);
-  a.Smax = static_cast<int>(Smax);
-  a.Hq = static_cast<int>(Hq);
-  a.Hkv = static_cast<int>(Hkv);
-  a.D = static_cast<int>(D);
-  a.W = window;
-  a.scale = scale;
-  const int64_t vis = window < Smax ? window : Smax;
-  if (chunk == 0) {
-    // keep every sequence within 32 splits (the exact small-split combine)
-    int64_t c = ((vis + 31) / 32 + 63) / 64 * 64;
-    chunk = static_cast<int32_t>(c < 256 ? 256 : c);
-  }
-  a.chunk = chunk;
-  for (int d = 0; d < 2; ++d) {
-    a.q_s[d] = q->stride[d];
-    a.o_s[d] = out->stride[d];
-  }
-  for (int d = 0; d < 3; ++d) {
-    a.kc_s[d] = kcache->stride[d];
-    a.vc_s[d] = vcache->stride[d];
-  }
+  bool empty;
+  int rc = prep_decode(q, kcache, vcache, seqlens, sinks, window, scale, chunk, out, &a, &empty);
+  if (rc || empty) return rc;
   if ((rc = status_ptr(&a.status))) return rc;
   cudaMemPool_t pool;
   if ((rc = workspace_pool(&pool))) return rc;

@@ -151,6 +151,19 @@ def test_decode_rejects_invalid_arguments(lib, case):
     assert rc == expect, (case, rc, abi.attn_sink_last_error())
 
 
+def test_noalloc_decode_rejects_workspace_beyond_its_array(lib):
+    """The no-allocation decode checks its workspace bound on the host and
+    refuses, with a message naming both sizes, before any device work."""
+    B, Smax, Hq, Hkv, D = 256, 131072, 32, 4, 128   # ~135 MB of workspace
+    q, o = _t([B, Hq, D]), _t([B, Hq, D])
+    kc = _t([B, Smax, Hkv, D])
+    sl, s = _t([B], abi.ATTN_DTYPE_I32), _t([Hq], abi.ATTN_DTYPE_F32)
+    r = ctypes.byref
+    rc = lib.attn_sink_decode_noalloc(r(q), r(kc), r(kc), r(sl), r(s), Smax, 0.125, r(o), None)
+    assert rc == abi.ATTN_EUNSUPPORTED
+    assert "workspace" in abi.attn_sink_last_error()
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(abi, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(abi, "_lib", None)
