@@ -8,21 +8,31 @@
 // its "fix 1" the rule for the TMEM allocation barrier (every warp that uses
 // TMEM takes part in it, and one constant defines that set).  The kernel
 // layout follows the FA4 SM100 design the flash-attention contributor-guide
-// page describes (load / MMA / softmax roles, S and O accumulated in TMEM) as
-// prior art; everything here is written for sm_100a directly.
+// page describes (load / MMA / softmax roles, S and O accumulated in TMEM,
+// two query tiles per CTA in ping-pong) as prior art; everything here is
+// written for sm_100a directly.
 //
-// One CTA computes one 128-row query tile of one head:
-//   warp 4      TMA producer: Q once, then K/V tiles into a ring of stages in
-//               the order the MMA warp consumes them (K0, K1, V0, K2, V1, ...)
-//   warp 5      TMEM allocator and MMA issuer: S_j = Q K_j^T into one of two
-//               TMEM S buffers, O += P_j V_j with P_j read from TMEM
-//   warps 0-3   softmax / correction / epilogue, one thread per query row
-//               (TMEM lane); P_j is written as bf16 over S_j's columns.
+// One CTA computes one 128-row query tile for NH query heads of the same
+// kv-head group (NH = 2 when the group size is even).  Those heads read the
+// same K/V tiles under the same mask, so every K/V tile brought from L2 feeds
+// NH x 128 query rows.  Warps:
+//   0 .. 4*NH-1  softmax / correction / epilogue: warpgroup w owns head slot
+//                w, one thread per query row (TMEM lane)
+//   4*NH         TMA producer: Q (NH tiles) once, then K_0, V_0, K_1, V_1, ...
+//                into a ring of shared-memory stages
+//   4*NH+1       TMEM allocator and MMA issuer, in the order
+//                S^0_0, S^1_0, then per key tile j:
+//                  PV^0_j, S^0_{j+1}, PV^1_j, S^1_{j+1}
+//                so that while one warpgroup exponentiates, the tensor cores
+//                work for the other (ping-pong).
+// TMEM (columns): S^w at w*BN (P^w written as bf16 over its first BN/2
+// columns), O^w at NH*BN + w*D.
 // Only the K tiles that meet the window [m0-W+1, m0+127] are visited; the
 // mask is applied on the tiles that cross the causal diagonal, the window's
 // lower edge or the end of the sequence.
 #include <math.h>
 
+#include "exp2_poly.h"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -30,46 +40,78 @@ namespace attnsink {
 namespace {
 
 constexpr int kBM = 128;             // query rows per tile (= TMEM lanes)
-constexpr int kSoftmaxWarps = 4;     // warps 0..3
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
-// The warps that touch TMEM: the softmax warpgroup and the MMA warp.  This is
-// the single definition of the TMEM allocation barrier's participant set; the
-// barrier count and the participation test below both derive from it.
-constexpr uint32_t kTmemWarpMask = 0x0Fu | (1u << kMmaWarp);
-constexpr uint32_t kTmemThreads = 32u * __builtin_popcount(kTmemWarpMask);
-__host__ __device__ constexpr bool is_tmem_warp(int w) { return (kTmemWarpMask >> w) & 1u; }
-
-constexpr uint32_t kBarTmem = 1;     // named barrier ids (0 = __syncthreads)
-constexpr uint32_t kBarEpilogue = 2;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kBarTmem = 1;     // named barrier ids (0 = __syncthreads);
+constexpr uint32_t kBarEpilogue0 = 2;  // 2 + w: epilogue of warpgroup w
 // Lazy rescaling: the running maximum (log2 units) only moves when a tile's
 // maximum exceeds it by more than this; until then exponents stay <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Of every 8 columns of P, this many take the FMA-pipe polynomial for 2^x and
+// the rest the MUFU ex2 (the two pipes then finish at about the same time).
+constexpr int kPolyPerOctet = 0;
+// Instruction mix of the exponentiation pass (chosen by measurement).
+constexpr bool kPackedFma = true;   // f32x2 FMA for S*scale*log2e - m
+constexpr bool kPackedAdd = true;   // f32x2 adds for the row sum
+constexpr bool kFusedMax = true;    // tile maximum in the same pass (else: sum test)
 
 // wait-location codes reported with ATTN_ETIMEOUT
 enum : int { kWhereQ = 101, kWhereFull = 102, kWhereEmpty = 103, kWhereS = 104, kWhereP = 105,
              kWhereO = 106 };
 
-template <int D, int BN>
+template <int D, int BN, int NH>
 struct Cfg {
+  static constexpr int kSoftmaxWarps = 4 * NH;
+  static constexpr int kProducerWarp = 4 * NH;
+  static constexpr int kMmaWarp = 4 * NH + 1;
+  // With two softmax warpgroups the producer and MMA warps are padded to a
+  // whole third warpgroup, which hands registers to the softmax warpgroups.
+  static constexpr int kWarps = NH == 2 ? 12 : 4 * NH + 2;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr bool kRealloc = NH == 2;
+  static constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 88;
+  static_assert(!kRealloc || (8 * kRegsSoftmax + 4 * kRegsOther) * 32 <= 65536 / kThreads / 8 * 8 * kThreads,
+                "register split exceeds the launch allocation");
+  // The warps that touch TMEM: the softmax warpgroups and the MMA warp.  This
+  // is the single definition of the TMEM allocation barrier's participant
+  // set; the barrier count and the participation test both derive from it.
+  static constexpr uint32_t kTmemWarpMask = ((1u << (4 * NH)) - 1u) | (1u << kMmaWarp);
+  static constexpr uint32_t kTmemThreads = 32u * __builtin_popcount(kTmemWarpMask);
+
   static constexpr int kChunks = D / 64;          // 64-channel (128-byte) column chunks
-  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kBarBytes = 512;           // mbarriers, TMEM base, abort flag
+  static constexpr int kQTileBytes = kBM * D * 2;
+  static constexpr int kQBufBytes = NH * kQTileBytes;   // one unit's Q tiles (later its O staging)
+  static constexpr int kQBytes = 2 * kQBufBytes;        // double buffered across units
   static constexpr int kTileBytes = BN * D * 2;   // one K or V tile
-  static constexpr int kStages = (D == 64) ? 8 : (D == 128 ? 5 : 4);
+  // S buffers per head: two (S_{j+1} computed while S_j is exponentiated)
+  // when TMEM has room, else one (the other head's work fills the gap)
+  static constexpr int kSBuf = NH * (2 * BN + D) <= 512 ? 2 : 1;
+  static constexpr int kColsUsed = NH * (kSBuf * BN + D);
+  static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256u : 512u;
+  static constexpr int kCtasPerSm = (kTmemCols == 256u) ? 2 : 1;
+  // per-CTA shared-memory budget: the SM's 228 KB shared by kCtasPerSm CTAs,
+  // each also reserving 1 KB, minus the barrier block and alignment slack
+  static constexpr int kBudget = (228 * 1024) / kCtasPerSm - 1024 - kBarBytes - 1024;
+  static constexpr int kStagesRaw = (kBudget - kQBytes) / kTileBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kRingBytes = kStages * kTileBytes;
   static constexpr int kBarOffset = kQBytes + kRingBytes;
-  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
-  static constexpr uint32_t kOCol = 2 * BN;                    // O accumulator column
-  static_assert(2 * BN + D <= (int)kTmemCols, "TMEM budget");
+  static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;  // + barriers + alignment slack
+  static constexpr uint32_t kSCol(int w, int buf) { return static_cast<uint32_t>((kSBuf * w + buf) * BN); }
+  static constexpr uint32_t kOCol(int w) { return static_cast<uint32_t>(kSBuf * NH * BN + w * D); }
+  static_assert(kStages >= 2, "need at least two ring stages");
+  static_assert(kColsUsed <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared-memory budget");
 };
 
+template <int D, int BN, int NH>
+__host__ __device__ constexpr bool is_tmem_warp(int w) {
+  return (Cfg<D, BN, NH>::kTmemWarpMask >> w) & 1u;
+}
+
 struct Params {
-  int L, Hq, W, group, num_m_tiles;
+  int L, Hq, W, group, num_m_tiles, B, num_units;
   float scale_log2;
   const float *sinks;
   float *lse;
@@ -94,84 +136,317 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// Columns outside [lo, hi] of a 32-column chunk starting at column c0 -> -inf.
+__device__ __forceinline__ void mask_chunk(uint32_t (&x)[32], int c0, int lo, int hi) {
+#pragma unroll
+  for (int t = 0; t < 32; ++t)
+    if (c0 + t < lo || c0 + t > hi) x[t] = __float_as_uint(-INFINITY);
+}
+
+__device__ __forceinline__ float max32(const uint32_t (&x)[32]) {
+  float a[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) a[u] = __uint_as_float(x[u]);
+#pragma unroll
+  for (int t = 4; t < 32; t += 4)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = fmaxf(a[u], __uint_as_float(x[t + u]));
+  return fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ void f2unpack(uint64_t r, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a packed pair on the FMA/ALU pipes (no MUFU).  Cody-Waite reduction
+// x = n + f, n = round(x) (via the 1.5*2^23 shifter), f in [-1/2, 1/2];
+// 2^f from the degree-3 fit of exp2_poly.h; 2^n added to the exponent field.
+// Inputs below -126 are clamped there (2^-126 ~ 1e-38 instead of 0).
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x, float &y0, float &y1) {
+  const float kShift = 12582912.0f;                // 1.5 * 2^23
+  float x0, x1;
+  f2unpack(x, x0, x1);
+  x = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = add2(x, f2pack(kShift, kShift));         // n in the low mantissa bits
+  const uint64_t nf = add2(t, f2pack(-kShift, -kShift));      // n as a float
+  const uint64_t f = add2(x, nf ^ 0x8000000080000000ull);     // x - n
+  uint64_t q = fma2(f, f2pack(kExp2C3, kExp2C3), f2pack(kExp2C2, kExp2C2));
+  q = fma2(q, f, f2pack(kExp2C1, kExp2C1));
+  q = fma2(q, f, f2pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(q0) + __float_as_uint(t0) * 8388608u);   // + n << 23
+  y1 = __uint_as_float(__float_as_uint(q1) + __float_as_uint(t1) * 8388608u);
+}
+
+// P = 2^(S*scale*log2e - m_use) for one row tile held in registers (sv),
+// written as bf16 over the first BN/2 columns at p_addr; returns the fp32 sum
+// of P, and with kMax also the tile's raw maximum in tmax.  Of every 8
+// columns kPolyPerOctet take the FMA-pipe polynomial for 2^x, the rest MUFU.
+template <int BN, bool kMax>
+__device__ __forceinline__ float exp_tile(const uint32_t (&sv)[BN / 32][32], uint32_t p_addr,
+                                          float sl2, float m_use, uint32_t cls_none, float &tmax) {
+  const uint64_t sl2x2 = f2pack(sl2, sl2);
+  const uint64_t negm2 = f2pack(-m_use, -m_use);
+  uint64_t acc2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+  float accs[4] = {0.f, 0.f, 0.f, 0.f};
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t pk[16];
+    if (cls_none >> c & 1u) {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) pk[t] = 0u;
+    } else {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const float s0 = __uint_as_float(sv[c][2 * t]), s1 = __uint_as_float(sv[c][2 * t + 1]);
+        if (kMax) mx[t & 3] = fmax3(mx[t & 3], s0, s1);
+        float z0, z1;
+        if (kPackedFma) {
+          f2unpack(fma2(f2pack(s0, s1), sl2x2, negm2), z0, z1);
+        } else {
+          z0 = fmaf(s0, sl2, -m_use);
+          z1 = fmaf(s1, sl2, -m_use);
+        }
+        float p0, p1;
+        if ((t & 3) < kPolyPerOctet / 2) {
+          exp2_poly_x2(f2pack(z0, z1), p0, p1);
+        } else {
+          p0 = ex2_approx(z0);
+          p1 = ex2_approx(z1);
+        }
+        if (kPackedAdd) {
+          acc2[t & 1] = add2(acc2[t & 1], f2pack(p0, p1));
+        } else {
+          accs[t & 3] += p0;
+          accs[(t + 2) & 3] += p1;
+        }
+        pk[t] = pack_bf16x2(p0, p1);
+      }
+    }
+    tmem_st16(p_addr + c * 16, pk);
+  }
+  if (kMax) tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  if (kPackedAdd) {
+    float a0, a1, b0, b1;
+    f2unpack(acc2[0], a0, a1);
+    f2unpack(acc2[1], b0, b1);
+    return (a0 + a1) + (b0 + b1);
+  }
+  return (accs[0] + accs[1]) + (accs[2] + accs[3]);
+}
+
+// Raw maximum of the non-empty chunks of a row tile held in registers.
+template <int BN>
+__device__ __forceinline__ float tile_max(const uint32_t (&sv)[BN / 32][32], uint32_t cls_none) {
+  float a[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) a[u] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    if (cls_none >> c & 1u) continue;
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      a[t & 7] = fmax3(a[t & 7], __uint_as_float(sv[c][2 * t]), __uint_as_float(sv[c][2 * t + 1]));
+  }
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// One key tile of the online softmax for the calling thread's row (its TMEM
+// lane): read S (one TMEM round trip), mask, update the running state and
+// write P over S.  From the second tile on, P is computed against the running
+// maximum while the tile maximum is found in the same pass; only if a row's
+// maximum then grew by more than the lazy-rescale threshold (rare after the
+// first tiles) does its warp rescale O and recompute P.  Returns false if a
+// bounded wait ran out.
 template <int D, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col, uint32_t o_col,
+                                             int j, int g, float sl2, int lo, int hi, uint32_t cls_mask,
+                                             uint32_t cls_none, float &m_run, float &l_run,
+                                             uint64_t *pv_done, const WaitCtx &ctx) {
+  constexpr int NC = BN / 32;
+  uint32_t sv[NC][32];
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (!(cls_none >> c & 1u)) tmem_ld32(lane_base + s_col + c * 32, sv[c]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (cls_mask >> c & 1u) mask_chunk(sv[c], c * 32, lo, hi);
+  float tm;
+  if (j == 0) {
+    // first tile: nothing accumulated yet, so take the maximum first
+    const float mt2 = tile_max<BN>(sv, cls_none) * sl2;
+    if (mt2 > m_run + kRescaleThreshold) m_run = mt2;
+    l_run = exp_tile<BN, false>(sv, lane_base + s_col, sl2, (m_run == -INFINITY) ? 0.f : m_run,
+                                cls_none, tm);
+    return true;
+  }
+  const float sum = exp_tile<BN, kFusedMax>(sv, lane_base + s_col, sl2,
+                                            (m_run == -INFINITY) ? 0.f : m_run, cls_none, tm);
+  // Without the fused maximum: every P <= 2^threshold when the tile's sum is
+  // at most that, so no row can have moved past the threshold; otherwise the
+  // maximum is taken now (and usually turns out not to have moved either).
+  if (!kFusedMax) tm = (sum <= 256.f) ? -INFINITY : tile_max<BN>(sv, cls_none);
+  const float mt2 = tm * sl2;
+  const bool grow = mt2 > m_run + kRescaleThreshold;
+  if (!__any_sync(0xffffffffu, grow)) {
+    l_run += sum;
+    return true;
+  }
+  // Rare path: some row's maximum moved.  O holds sum_{t<j} P_t V_t once
+  // PV_{j-1} has finished (S_j finished implies that the PVs issued before it,
+  // up to PV_{j-kSBuf}, finished, so the barrier is at most one phase behind
+  // and the parity wait is exact); rescale it and recompute P.
+  float alpha = 1.f;
+  if (grow) {
+    alpha = ex2_approx(m_run - mt2);               // 0 while nothing was seen yet
+    m_run = mt2;
+  }
+  if (!warp_wait(pv_done, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereO)) return false;
+  tc_fence_after();
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(lane_base + o_col + c * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+    tmem_st32(lane_base + o_col + c * 32, o);
+  }
+  tmem_wait_st();
+  l_run = l_run * alpha + exp_tile<BN, false>(sv, lane_base + s_col, sl2,
+                                              (m_run == -INFINITY) ? 0.f : m_run, cls_none, tm);
+  return true;
+}
+
+template <int D, int BN, int NH>
+__global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const Params p) {
-  using C = Cfg<D, BN>;
+  using C = Cfg<D, BN, NH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  uint8_t *sQ = smem;                       // Q tile, later the O staging tile
+  uint8_t *sQ = smem;                       // [2] units' Q tiles, later their O staging
   uint8_t *sRing = smem + C::kQBytes;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
   uint64_t *empty = full + C::kStages;
-  uint64_t *q_full = empty + C::kStages;
-  uint64_t *s_full = q_full + 1;            // [2]
-  uint64_t *p_full = s_full + 2;
-  uint64_t *o_full = p_full + 1;
-  uint64_t *mma_done = o_full + 1;
+  uint64_t *q_full = empty + C::kStages;    // [2] a unit's Q landed in buffer u%2
+  uint64_t *q_empty = q_full + 2;           // [2] buffer u%2's O store has read it (NH arrivals)
+  uint64_t *s_full = q_empty + 2;           // [NH][2] S^w ready in S buffer
+  uint64_t *p_full = s_full + 2 * NH;       // [NH][2] P^w ready in S buffer (O^w rescaled)
+  uint64_t *pv_done = p_full + 2 * NH;      // [NH] one PV^w finished
+  uint64_t *o_full = pv_done + NH;          // every MMA of a unit finished
+  uint64_t *o_drained = o_full + 1;         // [NH] O^w of a unit read out of TMEM
+  uint64_t *mma_done = o_drained + NH;      // every MMA of the CTA finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   const WaitCtx ctx{abort_flag, p.status};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Later query tiles see more keys under a causal window; launch them first.
-  const int mt = p.num_m_tiles - 1 - static_cast<int>(blockIdx.x);
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int hk = h / p.group;
-  const int m0 = mt * kBM;
-  const int row_last = min(p.L - 1, m0 + kBM - 1);
-  const int key_lo = max(0, m0 - p.W + 1);
-  const int kt0 = key_lo / BN;
-  const int n_tiles = row_last / BN - kt0 + 1;
+  const int HP = p.Hq / NH;                 // head groups (units per position and batch)
+  // Work units: (query tile, head group, batch), latest query tiles first (they
+  // see the most keys under a causal window), head groups fastest so that the
+  // CTAs running at the same time share K/V tiles in L2.  CTA c takes units
+  // c, c + gridDim.x, ...
+  struct Unit {
+    int m0, h0, b, kt0, n_tiles;
+  };
+  auto unit_at = [&](int u) {
+    Unit t;
+    const int per_m = HP * p.B;
+    const int mt = p.num_m_tiles - 1 - u / per_m;
+    const int r = u - (u / per_m) * per_m;
+    t.h0 = (r % HP) * NH;
+    t.b = r / HP;
+    t.m0 = mt * kBM;
+    const int row_last = min(p.L - 1, t.m0 + kBM - 1);
+    t.kt0 = max(0, t.m0 - p.W + 1) / BN;
+    t.n_tiles = row_last / BN - t.kt0 + 1;
+    return t;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, kSoftmaxWarps * 32);
+    for (int qb = 0; qb < 2; ++qb) {
+      mbar_init(&q_full[qb], 1);
+      mbar_init(&q_empty[qb], NH);
+    }
+    for (int w = 0; w < NH; ++w) {
+      for (int buf = 0; buf < 2; ++buf) {
+        mbar_init(&s_full[2 * w + buf], 1);
+        mbar_init(&p_full[2 * w + buf], 128);
+      }
+      mbar_init(&pv_done[w], 1);
+      mbar_init(&o_drained[w], 128);
+    }
     mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-
   // ---- TMEM allocation (page "cf-1.com/news/6055759", fix 1) ----
   // The MMA warp allocates; every TMEM warp then meets at one named barrier
   // whose count is exactly the number of threads in kTmemWarpMask, and only
   // after it reads the column base.
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   uint32_t tmem = 0;
-  if (is_tmem_warp(warp)) {
+  if (is_tmem_warp<D, BN, NH>(warp)) {
     tc_fence_before();
-    named_barrier_sync(kBarTmem, kTmemThreads);
+    named_barrier_sync(kBarTmem, C::kTmemThreads);
     tc_fence_after();
     tmem = *tmem_slot;
   }
 
-  if (warp == kProducerWarp) {
+  if (warp >= C::kSoftmaxWarps) {
+  // Producer/MMA warpgroup: hand registers to the softmax warpgroups (every
+  // warp of the warpgroup, the idle padding warps included, executes this).
+  if constexpr (C::kRealloc) setmaxnreg_dec<C::kRegsOther>();
+  if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_4d(sQ + c * kBM * 128, &tmQ, q_full, c * 64, h, m0, b);
-      int slot = 0;
+      int slot = 0, q_loaded = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap *map, int kt) {
+      auto load = [&](const CUtensorMap *map, int kt, int b) {
         const int s = slot % C::kStages;
         const uint32_t use = static_cast<uint32_t>(slot / C::kStages);
         if (slot >= C::kStages && !mbar_wait(&empty[s], (use & 1u) ^ 1u, ctx, kWhereEmpty)) {
@@ -181,31 +456,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], C::kTileBytes);
         uint8_t *dst = sRing + s * C::kTileBytes;
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(dst + c * BN * 128, map, &full[s], c * 64, hk, kt * BN, b);
+          tma_load_4d(dst + c * BN * 128, map, &full[s], c * 64, 0, kt * BN, b);
         ++slot;
       };
-      load(&tmK, kt0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles) load(&tmK, kt0 + j + 1);
-        if (ok) load(&tmV, kt0 + j);
+      for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; ++ul, u += gridDim.x) {
+        const Unit t = unit_at(u);
+        const int qb = ul & 1;
+        // the buffer's previous unit has stored its O out of it
+        if (ul >= 2 &&
+            !mbar_wait(&q_empty[qb], static_cast<uint32_t>((ul >> 1) - 1) & 1u, ctx, kWhereQ)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[qb], C::kQBufBytes);
+        for (int w = 0; w < NH; ++w)
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sQ + qb * C::kQBufBytes + w * C::kQTileBytes + c * kBM * 128, &tmQ,
+                        &q_full[qb], c * 64, t.h0 + w, t.m0, t.b);
+        q_loaded = ul + 1;
+        const int hk = t.h0 / p.group;
+        // the order the MMA warp consumes: K_0 .. K_{kSBuf-1}, then per tile
+        // j: V_j, K_{j+kSBuf}
+        auto kv = [&](const CUtensorMap *map, int kt) {
+          const int s = slot % C::kStages;
+          const uint32_t use = static_cast<uint32_t>(slot / C::kStages);
+          if (slot >= C::kStages && !mbar_wait(&empty[s], (use & 1u) ^ 1u, ctx, kWhereEmpty)) {
+            ok = false;
+            return;
+          }
+          mbar_arrive_expect_tx(&full[s], C::kTileBytes);
+          uint8_t *dst = sRing + s * C::kTileBytes;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(dst + c * BN * 128, map, &full[s], c * 64, hk, kt * BN, t.b);
+          ++slot;
+        };
+        for (int jj = 0; ok && jj < C::kSBuf && jj < t.n_tiles; ++jj) kv(&tmK, t.kt0 + jj);
+        for (int j = 0; ok && j < t.n_tiles; ++j) {
+          kv(&tmV, t.kt0 + j);
+          if (ok && j + C::kSBuf < t.n_tiles) kv(&tmK, t.kt0 + j + C::kSBuf);
+        }
       }
+      (void)load;
       if (!ok) {
         // Leaving early: let the copies already issued land before the CTA
         // (and its shared memory) goes away.
-        drain_wait(q_full, 0);
+        if (q_loaded > 0)
+          drain_wait(&q_full[(q_loaded - 1) & 1], static_cast<uint32_t>((q_loaded - 1) >> 1) & 1u);
         for (int t = max(0, slot - C::kStages); t < slot; ++t)
           drain_wait(&full[t % C::kStages], static_cast<uint32_t>(t / C::kStages) & 1u);
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == C::kMmaWarp) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(kBM, BN, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_pv = umma_idesc_bf16(kBM, D, 0, 1);   // V is N-major
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t ring_base = smem_u32(sRing);
-      bool ok = mbar_wait(q_full, 0, ctx, kWhereQ);
+      // descriptor words: 128-byte swizzle, 8-row groups 1024 bytes apart;
+      // K-major operands (Q, K) need no leading offset, the N-major V tile has
+      // its 64-channel chunks BN*128 bytes apart
+      const uint32_t desc_hi = umma_desc_hi_sw128(1024);
+      const uint32_t q_lo = umma_desc_lo(smem_u32(sQ), 16);
+      const uint32_t ring_lo_k = umma_desc_lo(smem_u32(sRing), 16);
+      const uint32_t ring_lo_v = umma_desc_lo(smem_u32(sRing), BN * 128);
+      bool ok = true;
       int slot = 0;
       auto acquire = [&](int &s) {
         s = slot % C::kStages;
@@ -215,191 +529,216 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return ok;
       };
-      auto issue_s = [&](int j, int s) {
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>((j & 1) * BN);
-        const uint32_t k_base = ring_base + s * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;   // 16 channels = 32 bytes along the row
-          const uint64_t a = umma_smem_desc_sw128(q_base + (kk >> 2) * (kBM * 128) + koff, 16, 1024);
-          const uint64_t bd = umma_smem_desc_sw128(k_base + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-          umma_ss(d_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+      int jg = 0;                            // tiles of earlier units (barrier phases)
+      for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; ++ul, u += gridDim.x) {
+        const Unit t = unit_at(u);
+        const int qb = ul & 1;
+        if (!mbar_wait(&q_full[qb], static_cast<uint32_t>(ul >> 1) & 1u, ctx, kWhereQ)) {
+          ok = false;
+          break;
         }
-        umma_commit(&s_full[j & 1]);
-        umma_commit(&empty[s]);
-      };
-      auto issue_pv = [&](int j, int s) {
-        const uint32_t a_tmem = tmem + static_cast<uint32_t>((j & 1) * BN);
-        const uint32_t v_base = ring_base + s * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = umma_smem_desc_sw128(v_base + kk * 16 * 128, BN * 128, 1024);
-          umma_ts(tmem + C::kOCol, a_tmem + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(o_full);
-        umma_commit(&empty[s]);
-      };
-      int s;
-      if (ok && acquire(s)) issue_s(0, s);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles) {
-          if (!acquire(s)) break;
-          issue_s(j + 1, s);
-        }
-        if (!mbar_wait(p_full, static_cast<uint32_t>(j) & 1u, ctx, kWhereP)) break;
         tc_fence_after();
-        if (!acquire(s)) break;
-        issue_pv(j, s);
+        // S^w_j = Q^w K_j^T into S buffer (jg+j)%kSBuf of head w (overwriting
+        // the P^w that the PV^w issued before it has consumed: the tensor pipe
+        // runs in order)
+        auto issue_s = [&](int w, int ks, int j) {
+          const int g = jg + j;
+          const uint32_t a0 = q_lo + ((qb * C::kQBufBytes + w * C::kQTileBytes) >> 4);
+          const uint32_t b0 = ring_lo_k + ks * (C::kTileBytes >> 4);
+          const uint32_t d = tmem + C::kSCol(w, g % C::kSBuf);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
+            umma_ss_w(d, a0 + (kk >> 2) * (kBM * 128 >> 4) + (kk & 3) * 2, desc_hi,
+                      b0 + (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2, desc_hi, idesc_qk,
+                      kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[2 * w + g % C::kSBuf]);
+        };
+        // O^w += P^w_j V_j with P^w_j (bf16 pairs) in the first BN/2 columns
+        // of its S buffer
+        auto issue_pv = [&](int w, int vs, int j) {
+          const int g = jg + j;
+          const uint32_t b0 = ring_lo_v + vs * (C::kTileBytes >> 4);
+          const uint32_t a0 = tmem + C::kSCol(w, g % C::kSBuf);
+          const uint32_t d = tmem + C::kOCol(w);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts_w(d, a0 + kk * 8, b0 + kk * (16 * 128 >> 4), desc_hi, idesc_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&pv_done[w]);
+        };
+        int ks = 0, vs = 0;
+        for (int jj = 0; ok && jj < C::kSBuf && jj < t.n_tiles; ++jj) {
+          if (!acquire(ks)) break;
+          for (int w = 0; w < NH; ++w) issue_s(w, ks, jj);
+          umma_commit(&empty[ks]);
+        }
+        for (int j = 0; ok && j < t.n_tiles; ++j) {
+          const int g = jg + j;
+          const bool more = j + C::kSBuf < t.n_tiles;
+          if (!acquire(vs)) break;
+          for (int w = 0; w < NH; ++w) {
+            if (!mbar_wait(&p_full[2 * w + g % C::kSBuf], static_cast<uint32_t>(g / C::kSBuf) & 1u,
+                           ctx, kWhereP)) {
+              ok = false;
+              break;
+            }
+            // the first PV of a unit overwrites O^w: the previous unit's O^w
+            // must have been read out of TMEM
+            if (j == 0 && ul > 0 &&
+                !mbar_wait(&o_drained[w], static_cast<uint32_t>(ul - 1) & 1u, ctx, kWhereO)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(w, vs, j);
+            if (w == NH - 1) umma_commit(&empty[vs]);
+            if (more) {
+              if (w == 0 && !acquire(ks)) break;
+              issue_s(w, ks, j + C::kSBuf);
+              if (w == NH - 1) umma_commit(&empty[ks]);
+            }
+          }
+        }
+        jg += t.n_tiles;
+        umma_commit(o_full);                 // this unit's O is complete
       }
       // Every tensor-core operation of this CTA has finished before teardown.
       umma_commit(mma_done);
       drain_wait(mma_done, 0);
     }
     __syncwarp();
+    // ---- teardown: all TMEM users are done before the allocator frees it ----
+    tc_fence_before();
+    named_barrier_sync(kBarTmem, C::kTmemThreads);
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
   } else {
+    if constexpr (C::kRealloc) setmaxnreg_inc<C::kRegsSoftmax>();
     // ------------------------------------------- softmax / correction / epilogue
-    const int r = threadIdx.x;                       // tile row == TMEM lane
-    const int i = m0 + r;                            // query position
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int w = warp >> 2;                         // head slot of this warpgroup
+    const int r = threadIdx.x & 127;                 // tile row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t o_col = C::kOCol(w);
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;                         // running max, log2 units
-    float l_run = 0.f;                               // running denominator
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!warp_wait(&s_full[j & 1], static_cast<uint32_t>(j >> 1) & 1u, ctx, kWhereS)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t s_addr = lane_base + static_cast<uint32_t>((j & 1) * BN);
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(s_addr + c * 32, raw);
-        tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 32; ++t) s[c * 32 + t] = __uint_as_float(raw[t]);
-      }
-      const int kbase = (kt0 + j) * BN;
-      // Tile-uniform test: does any (row, key) of this tile fall outside the
-      // causal window or past the end of the sequence?
-      const bool edge = (kbase + BN - 1 > m0) || (kbase < m0 + kBM - p.W) || (kbase + BN > p.L);
-      if (edge) {
-        const int lo = i - p.W + 1 - kbase;          // first visible column
-        const int hi = min(i, p.L - 1) - kbase;      // last visible column
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c < lo || c > hi) s[c] = -INFINITY;
-      }
-      float mt = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mt = fmaxf(mt, s[c]);
-      const float mt2 = mt * sl2;
-      float alpha = 1.f;
-      if (mt2 > m_run + kRescaleThreshold) {
-        alpha = ex2_approx(m_run - mt2);             // 0 while nothing was seen yet
-        m_run = mt2;
-      }
-      l_run *= alpha;
-      if (j > 0) {
-        // O holds sum_{t<j} P_t V_t: wait for PV_{j-1}, then rescale it if
-        // any row of this warp moved its maximum.
-        if (!warp_wait(o_full, static_cast<uint32_t>(j - 1) & 1u, ctx, kWhereO)) {
+    int jg = 0;
+    int pending_qb = -1;                             // buffer whose O store may still read it
+    for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; ++ul, u += gridDim.x) {
+      const Unit t = unit_at(u);
+      const int qb = ul & 1;
+      const int h = t.h0 + w;
+      const int i = t.m0 + r;                        // query position
+      float m_run = -INFINITY;                       // running max, log2 units
+      float l_run = 0.f;                             // running denominator
+      for (int j = 0; j < t.n_tiles; ++j) {
+        const int g = jg + j;
+        const uint32_t s_col = C::kSCol(w, g % C::kSBuf);
+        if (!warp_wait(&s_full[2 * w + g % C::kSBuf], static_cast<uint32_t>(g / C::kSBuf) & 1u,
+                       ctx, kWhereS)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + C::kOCol + c * 32, o);
-            tmem_wait_ld();
+        const int kbase = (t.kt0 + j) * BN;
+        // Tile-uniform test: does any (row, key) of this tile fall outside the
+        // causal window or past the end of the sequence?
+        const bool edge = (kbase + BN - 1 > t.m0) || (kbase < t.m0 + kBM - p.W) || (kbase + BN > p.L);
+        const int lo = i - p.W + 1 - kbase;          // first visible column
+        const int hi = min(i, p.L - 1) - kbase;      // last visible column
+        // Per 32-column chunk, a warp-uniform class: every lane's visible
+        // interval [lo, hi] covers the chunk (no mask), misses it (no work:
+        // P = 0), or cuts it (per-element mask).
+        uint32_t cls_mask = 0, cls_none = 0;         // bit c: chunk c mixed / empty
+        if (edge) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-            tmem_st32(lane_base + C::kOCol + c * 32, o);
+          for (int c = 0; c < BN / 32; ++c) {
+            const bool all_in = __all_sync(0xffffffffu, lo <= c * 32 && hi >= c * 32 + 31);
+            const bool all_out = __all_sync(0xffffffffu, hi < c * 32 || lo > c * 32 + 31);
+            cls_none |= (all_out ? 1u : 0u) << c;
+            cls_mask |= (!all_in && !all_out ? 1u : 0u) << c;
           }
         }
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * t], sl2, -m_use));
-          const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * t + 1], sl2, -m_use));
-          sum += p0 + p1;
-          pk[t] = pack_bf16x2(p0, p1);
+        if (!softmax_tile<D, BN>(lane_base, s_col, o_col, j, g, sl2, lo, hi, cls_mask, cls_none,
+                                 m_run, l_run, &pv_done[w], ctx)) {
+          ok = false;
+          break;
         }
-        tmem_st16(s_addr + c * 16, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * w + g % C::kSBuf]);
+        if (j == 0 && pending_qb >= 0 && r == 0) {
+          // The previous unit's O store has long finished reading its staging
+          // tile: hand the buffer back for the Q of a later unit.
+          tma_store_wait_read();
+          mbar_arrive(&q_empty[pending_qb]);
+          pending_qb = -1;
+        }
       }
-      l_run += sum;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    if (ok) ok = warp_wait(o_full, static_cast<uint32_t>(n_tiles - 1) & 1u, ctx, kWhereO);
-    tc_fence_after();
+      jg += t.n_tiles;
+      if (ok) ok = warp_wait(o_full, static_cast<uint32_t>(ul) & 1u, ctx, kWhereO);
+      if (!ok) break;
+      tc_fence_after();
+      // ---- sink epilogue (page "cf-1.com/news/6055759", fix 2) ----
+      // new = max(row max, sink*log2e); r = 2^(old-new);
+      // denominator' = denominator*r + 2^(sink*log2e - new); O = O_acc * r / denominator'.
+      const float sink2 = p.sinks[h] * kLog2e;
+      const float new_m = fmaxf(m_run, sink2);
+      const float rs = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - new_m);
+      const float l2 = l_run * rs + ((sink2 == -INFINITY) ? 0.f : ex2_approx(sink2 - new_m));
+      const float oscale = (l2 > 0.f) ? rs / l2 : 0.f;
+      const float lse_val = (l2 > 0.f) ? (new_m + log2f(l2)) * kLn2 : -INFINITY;
 
-    // ---- sink epilogue (page "cf-1.com/news/6055759", fix 2) ----
-    // new = max(row max, sink*log2e); r = 2^(old-new);
-    // denominator' = denominator*r + 2^(sink*log2e - new); O = O_acc * r / denominator'.
-    const float sink2 = p.sinks[h] * kLog2e;
-    const float new_m = fmaxf(m_run, sink2);
-    const float rs = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - new_m);
-    const float l2 = l_run * rs + ((sink2 == -INFINITY) ? 0.f : ex2_approx(sink2 - new_m));
-    const float oscale = (l2 > 0.f) ? rs / l2 : 0.f;
-    const float lse_val = (l2 > 0.f) ? (new_m + log2f(l2)) * kLn2 : -INFINITY;
-
-    if (ok) {
-      // O (fp32, TMEM) -> bf16 -> swizzled staging tile in the Q buffer ->
-      // TMA store; rows past the end of the sequence are clipped by the unit.
+      // O^w (fp32, TMEM) -> bf16 -> swizzled staging tile (this unit's Q^w
+      // buffer, no longer read) -> TMA store; rows past the end of the
+      // sequence are clipped.  Once O^w is out of TMEM the next unit's PV^w
+      // may overwrite it.
+      uint8_t *stage = sQ + qb * C::kQBufBytes + w * C::kQTileBytes;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(lane_base + C::kOCol + c * 32, o);
+        tmem_ld32(lane_base + o_col + c * 32, o);
         tmem_wait_ld();
-        uint8_t *chunk = sQ + (c >> 1) * (kBM * 128) + r * 128;
+        uint8_t *chunk = stage + (c >> 1) * (kBM * 128) + r * 128;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int uu = 0; uu < 4; ++uu) {
           uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * oscale, __uint_as_float(o[8 * u + 1]) * oscale);
-          v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * oscale, __uint_as_float(o[8 * u + 3]) * oscale);
-          v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * oscale, __uint_as_float(o[8 * u + 5]) * oscale);
-          v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * oscale, __uint_as_float(o[8 * u + 7]) * oscale);
-          const int unit = (c & 1) * 4 + u;          // 16-byte unit within the 128-byte row
+          v.x = pack_bf16x2(__uint_as_float(o[8 * uu + 0]) * oscale, __uint_as_float(o[8 * uu + 1]) * oscale);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * uu + 2]) * oscale, __uint_as_float(o[8 * uu + 3]) * oscale);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * uu + 4]) * oscale, __uint_as_float(o[8 * uu + 5]) * oscale);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * uu + 6]) * oscale, __uint_as_float(o[8 * uu + 7]) * oscale);
+          const int unit = (c & 1) * 4 + uu;        // 16-byte unit within the 128-byte row
           *reinterpret_cast<uint4 *>(chunk + ((unit ^ (r & 7)) << 4)) = v;
         }
       }
+      tc_fence_before();
+      mbar_arrive(&o_drained[w]);
       fence_proxy_async_smem();
+      if (w == 0)
+        named_barrier_sync(kBarEpilogue0, 128);
+      else
+        named_barrier_sync(kBarEpilogue0 + 1, 128);
+      if (r == 0) {
+        for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, stage + c * kBM * 128, c * 64, h, t.m0, t.b);
+        tma_store_commit();
+        pending_qb = qb;
+      }
+      if (p.lse != nullptr && i < p.L)
+        p.lse[static_cast<int64_t>(t.b) * p.lse_sb + static_cast<int64_t>(h) * p.lse_sh + i] = lse_val;
     }
-    named_barrier_sync(kBarEpilogue, kSoftmaxWarps * 32);
-    if (threadIdx.x == 0 && !*abort_flag) {
-      for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, sQ + c * kBM * 128, c * 64, h, m0, b);
-      tma_store_commit();
-      tma_store_wait_all();
-    }
-    if (ok && p.lse != nullptr && i < p.L)
-      p.lse[static_cast<int64_t>(b) * p.lse_sb + static_cast<int64_t>(h) * p.lse_sh + i] = lse_val;
-  }
-
-  // ---- teardown: all TMEM users are done before the allocator frees it ----
-  if (is_tmem_warp(warp)) {
+    // stores must have read shared memory before the CTA leaves
+    if (r == 0) tma_store_wait_all();
+    // teardown: this warp's TMEM reads are complete before the allocator frees it
     tc_fence_before();
-    named_barrier_sync(kBarTmem, kTmemThreads);
-    if (warp == kMmaWarp) {
-      tc_fence_after();
-      tmem_dealloc(tmem, kTmemCols);
-    }
+    named_barrier_sync(kBarTmem, C::kTmemThreads);
   }
 }
 
-template <int D, int BN>
+template <int D, int BN, int NH>
 cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
-  using C = Cfg<D, BN>;
+  using C = Cfg<D, BN, NH>;
   alignas(64) CUtensorMap mq, mk, mv, mo;
   cudaError_t e;
   if ((e = make_tma_bshd(&mq, a.q, a.B, a.L, a.Hq, D, a.q_s, kBM)) != cudaSuccess) return e;
@@ -412,28 +751,45 @@ cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
   p.W = a.W;
   p.group = a.Hq / a.Hkv;
   p.num_m_tiles = (a.L + kBM - 1) / kBM;
+  p.B = a.B;
+  p.num_units = p.num_m_tiles * (a.Hq / NH) * a.B;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.sinks = a.sinks;
   p.lse = a.lse;
   p.lse_sb = a.lse_s[0];
   p.lse_sh = a.lse_s[1];
   p.status = a.status;
-  auto kern = fwd_tc_kernel<D, BN>;
-  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                C::kSmemBytes)) != cudaSuccess)
-    return e;
-  dim3 grid(p.num_m_tiles, a.Hq, a.B);
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+  auto kern = fwd_tc_kernel<D, BN, NH>;
+  static bool attr_set[64] = {};  // once per device
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::kSmemBytes)) != cudaSuccess)
+      return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  static int sm_count[64] = {};
+  if (dev >= 0 && dev < 64 && sm_count[dev] == 0)
+    if ((e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+  const int sms = (dev >= 0 && dev < 64) ? sm_count[dev] : 148;
+  const int slots = sms * C::kCtasPerSm;
+  dim3 grid(p.num_units < slots ? p.num_units : slots);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream) {
+  // Two query heads per CTA when they share a kv head (even group size) and
+  // their S and O fit TMEM together; otherwise one.
+  const bool pair = (a.Hq / a.Hkv) % 2 == 0;
   switch (a.D) {
-    case 64: return launch<64, 128>(a, stream);
-    case 128: return launch<128, 128>(a, stream);
-    case 256: return launch<256, 64>(a, stream);
+    case 64: return pair ? launch<64, 128, 2>(a, stream) : launch<64, 64, 1>(a, stream);
+    case 128: return pair ? launch<128, 128, 2>(a, stream) : launch<128, 64, 1>(a, stream);
+    case 256: return launch<256, 64, 1>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
