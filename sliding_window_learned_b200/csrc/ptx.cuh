@@ -59,23 +59,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  Polls the barrier; every
-// 64 polls it checks the CTA abort flag and the elapsed time.  On timeout it
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or `hint_ns` pass, instead of returning at once: a waiting warp
+// then takes no issue slots from the warps doing work on its SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Longest time a waiting thread sleeps before it looks at the abort flag and
+// the elapsed time again.
+constexpr uint32_t kWaitSleepNs = 50000;
+
+// Bounded wait for the phase with the given parity.  The thread sleeps in the
+// barrier (woken when the phase completes); each time it wakes without the
+// phase it checks the CTA abort flag and the elapsed time.  On timeout it
 // records ATTN_ETIMEOUT (with `where` as the location code), raises the abort
 // flag so that the rest of the CTA stops waiting too, and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtx &ctx,
                                           int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*ctx.abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        report_timeout(ctx.status, where);
-        *ctx.abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (*ctx.abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      report_timeout(ctx.status, where);
+      *ctx.abort = 1;
+      return false;
     }
   }
 }
