@@ -83,14 +83,25 @@ def load() -> ctypes.CDLL:
     return _lib
 
 
+_DESC_CACHE: dict = {}
+
+
 def describe(t: torch.Tensor | None):
-    """An attn_tensor describing a torch tensor (None -> NULL)."""
+    """An attn_tensor describing a torch tensor (None -> NULL).  Descriptions
+    are cached by (address, dtype, shape, strides): a struct holds no more than
+    those, so a cached one is exact for any tensor with the same key."""
     if t is None:
         return None
+    key = (t.data_ptr(), t.dtype, tuple(t.shape), t.stride())
+    d = _DESC_CACHE.get(key)
+    if d is not None:
+        return d
     if t.dtype not in _DTYPES:
         raise TypeError(f"unsupported dtype {t.dtype}")
     if t.dim() > 4:
         raise ValueError("at most 4 dimensions")
+    if len(_DESC_CACHE) > 256:
+        _DESC_CACHE.clear()
     d = AttnTensor()
     d.data = t.data_ptr() if t.numel() > 0 else None
     d.dtype = _DTYPES[t.dtype]
@@ -98,6 +109,7 @@ def describe(t: torch.Tensor | None):
     for i in range(t.dim()):
         d.shape[i] = t.shape[i]
         d.stride[i] = t.stride(i)
+    _DESC_CACHE[key] = d
     return d
 
 

@@ -189,7 +189,32 @@ int prep_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
 }  // namespace
 
 // TMA descriptor for a [d3, d2, d1, d0] bf16 tensor, box {64, 1, box_rows, 1},
-// 128-byte swizzle, zero fill out of range.
+// 128-byte swizzle, zero fill out of range.  Encoded descriptors are kept in
+// a small least-recently-used cache keyed by everything that determines them
+// (address, sizes, strides, box), so repeated calls on the same buffers skip
+// the driver call.
+namespace {
+struct TmaKey {
+  const void *base;
+  int64_t d[4], s[3];
+  int box;
+  bool operator==(const TmaKey &o) const {
+    return base == o.base && box == o.box && memcmp(d, o.d, sizeof d) == 0 &&
+           memcmp(s, o.s, sizeof s) == 0;
+  }
+};
+struct TmaEntry {
+  TmaKey key;
+  alignas(64) CUtensorMap map;
+  uint64_t used;
+  bool valid;
+};
+constexpr int kTmaCacheSize = 64;
+TmaEntry g_tma_cache[kTmaCacheSize];
+uint64_t g_tma_tick = 0;
+std::mutex g_tma_mu;
+}  // namespace
+
 cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
                           int64_t d0, const int64_t strides_el[3], int box_rows) {
   typedef CUresult (*encode_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -207,6 +232,25 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
       encode = reinterpret_cast<encode_fn>(fn);
   });
   if (!encode) return cudaErrorNotSupported;
+  TmaKey key;
+  key.base = base;
+  key.d[0] = d0;
+  key.d[1] = d1;
+  key.d[2] = d2;
+  key.d[3] = d3;
+  key.s[0] = strides_el[0];
+  key.s[1] = strides_el[1];
+  key.s[2] = strides_el[2];
+  key.box = box_rows;
+  {
+    std::lock_guard<std::mutex> lk(g_tma_mu);
+    for (TmaEntry &e : g_tma_cache)
+      if (e.valid && e.key == key) {
+        e.used = ++g_tma_tick;
+        memcpy(map_out, &e.map, sizeof(CUtensorMap));
+        return cudaSuccess;
+      }
+  }
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
                               static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
   // byte strides of dims 1..3 (innermost first): head, position, batch
@@ -215,11 +259,27 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
                                  static_cast<cuuint64_t>(strides_el[0]) * 2};
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = encode(static_cast<CUtensorMap *>(map_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                            const_cast<void *>(base), dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  alignas(64) CUtensorMap map;
+  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  memcpy(map_out, &map, sizeof(CUtensorMap));
+  std::lock_guard<std::mutex> lk(g_tma_mu);
+  TmaEntry *victim = &g_tma_cache[0];
+  for (TmaEntry &e : g_tma_cache) {
+    if (!e.valid) {
+      victim = &e;
+      break;
+    }
+    if (e.used < victim->used) victim = &e;
+  }
+  victim->key = key;
+  memcpy(&victim->map, &map, sizeof(CUtensorMap));
+  victim->used = ++g_tma_tick;
+  victim->valid = true;
+  return cudaSuccess;
 }
 
 // Validates the decode arguments and fills `out_args`; `*empty` is set when
