@@ -57,7 +57,7 @@ constexpr bool kFusedMax = true;    // tile maximum in the same pass (else: sum 
 
 // wait-location codes reported with ATTN_ETIMEOUT
 enum : int { kWhereQ = 101, kWhereFull = 102, kWhereEmpty = 103, kWhereS = 104, kWhereP = 105,
-             kWhereO = 106, kWhereTurn = 107 };
+             kWhereO = 106 };
 
 template <int D, int BN, int NH>
 struct Cfg {
@@ -69,7 +69,7 @@ struct Cfg {
   static constexpr int kWarps = NH == 2 ? 12 : 4 * NH + 2;
   static constexpr int kThreads = kWarps * 32;
   static constexpr bool kRealloc = NH == 2;
-  static constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 88;
+  static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
   static_assert(!kRealloc || (8 * kRegsSoftmax + 4 * kRegsOther) * 32 <= 65536 / kThreads / 8 * 8 * kThreads,
                 "register split exceeds the launch allocation");
   // The warps that touch TMEM: the softmax warpgroups and the MMA warp.  This
@@ -278,27 +278,6 @@ __device__ __forceinline__ float tile_max(const uint32_t (&sv)[BN / 32][32], uin
   return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
 }
 
-// Alternation of the exponentiation passes of the two softmax warpgroups.
-// Both warpgroups share the SM's MUFU units; running their passes at the
-// same time only makes both take twice as long while the tensor cores wait
-// for their P.  So warpgroup 1's pass for tile g waits for warpgroup 0's pass
-// for tile g, and warpgroup 0's pass for tile g+1 waits for warpgroup 1's for
-// tile g (turn barriers, 128 arrivals each; S loads, P stores and the MMA
-// hand-offs still overlap the other warpgroup's pass).
-struct ExpTurn {
-  uint64_t *wait_bar;      // null: no wait for this tile
-  uint32_t wait_parity;
-  uint64_t *pass_bar;      // null: single warpgroup
-  __device__ __forceinline__ bool wait(const WaitCtx &ctx) const {
-    if (wait_bar == nullptr) return true;
-    const bool r = mbar_wait(wait_bar, wait_parity, ctx, kWhereTurn);
-    return __all_sync(0xffffffffu, r);
-  }
-  __device__ __forceinline__ void pass() const {
-    if (pass_bar != nullptr) mbar_arrive(pass_bar);
-  }
-};
-
 // One key tile of the online softmax for the calling thread's row (its TMEM
 // lane): read S (one TMEM round trip), mask, update the running state and
 // write P over S.  From the second tile on, P is computed against the running
@@ -310,7 +289,7 @@ template <int D, int BN>
 __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col, uint32_t o_col,
                                              int j, int g, float sl2, int lo, int hi, uint32_t cls_mask,
                                              uint32_t cls_none, float &m_run, float &l_run,
-                                             uint64_t *pv_done, const ExpTurn &turn,
+                                             uint64_t *pv_done,
                                              const WaitCtx &ctx) {
   constexpr int NC = BN / 32;
   uint32_t sv[NC][32];
@@ -326,16 +305,12 @@ __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col,
     // first tile: nothing accumulated yet, so take the maximum first
     const float mt2 = tile_max<BN>(sv, cls_none) * sl2;
     if (mt2 > m_run + kRescaleThreshold) m_run = mt2;
-    if (!turn.wait(ctx)) return false;
     l_run = exp_tile<BN, false>(sv, lane_base + s_col, sl2, (m_run == -INFINITY) ? 0.f : m_run,
                                 cls_none, tm);
-    turn.pass();
     return true;
   }
-  if (!turn.wait(ctx)) return false;
   const float sum = exp_tile<BN, kFusedMax>(sv, lane_base + s_col, sl2,
                                             (m_run == -INFINITY) ? 0.f : m_run, cls_none, tm);
-  turn.pass();
   // Without the fused maximum: every P <= 2^threshold when the tile's sum is
   // at most that, so no row can have moved past the threshold; otherwise the
   // maximum is taken now (and usually turns out not to have moved either).
@@ -393,8 +368,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   uint64_t *o_full = pv_done + NH;          // every MMA of a unit finished
   uint64_t *o_drained = o_full + 1;         // [NH] O^w of a unit read out of TMEM
   uint64_t *mma_done = o_drained + NH;      // every MMA of the CTA finished
-  uint64_t *turn = mma_done + 1;            // [2] exponentiation turns (two warpgroups)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(turn + 2);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   const WaitCtx ctx{abort_flag, p.status};
 
@@ -441,8 +415,6 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
     }
     mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
-    mbar_init(&turn[0], 128);
-    mbar_init(&turn[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -690,16 +662,8 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
             cls_mask |= (!all_in && !all_out ? 1u : 0u) << c;
           }
         }
-        ExpTurn et{nullptr, 0u, nullptr};
-        if (NH == 2) {
-          // warpgroup 1 follows warpgroup 0 on tile g; warpgroup 0 follows
-          // warpgroup 1 on tile g-1
-          if (w == 1) et.wait_bar = &turn[0], et.wait_parity = static_cast<uint32_t>(g) & 1u;
-          else if (g > 0) et.wait_bar = &turn[1], et.wait_parity = static_cast<uint32_t>(g - 1) & 1u;
-          et.pass_bar = &turn[w];
-        }
         if (!softmax_tile<D, BN>(lane_base, s_col, o_col, j, g, sl2, lo, hi, cls_mask, cls_none,
-                                 m_run, l_run, &pv_done[w], et, ctx)) {
+                                 m_run, l_run, &pv_done[w], ctx)) {
           ok = false;
           break;
         }
