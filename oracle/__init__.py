@@ -55,6 +55,8 @@ def _load():
         lib.oracle_fwd_rows.restype = I
         lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P]
         lib.oracle_decode.restype = I
+        lib.oracle_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P]
+        lib.oracle_decode_paged.restype = I
         lib.oracle_split_partial.argtypes = [P, P, P, ctypes.c_int64, I, I, I, F, P, P]
         lib.oracle_split_partial.restype = I
         lib.oracle_combine.argtypes = [I, P, P, I, F, P, P]
@@ -137,6 +139,32 @@ def decode(q, kcache, vcache, seqlens, sinks, window: int, scale: float):
                                float(scale), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_decode: invalid sizes")
+    return out, lse
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, sinks, window: int, scale: float):
+    """Single-token decode over a paged KV cache (see oracle.c).
+
+    q [B,Hq,D]; kpages/vpages [NB,P,Hkv,D] uint16 bf16 bits; block_table
+    [B,MP] int32 (position t of sequence b is row t % P of page
+    block_table[b, t // P]; entries outside [0, NB) are pages of zero rows);
+    seqlens [B] int32 in [0, MP*P]; sinks [Hq] float32.
+    Returns (out [B,Hq,D], lse [B,Hq]) float64."""
+    q, kpages, vpages, sinks = _u16(q), _u16(kpages), _u16(vpages), _f32(sinks)
+    block_table = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    seqlens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    B, Hq, D = q.shape
+    NB, P, Hkv, _ = kpages.shape
+    MP = block_table.shape[1]
+    assert kpages.shape == (NB, P, Hkv, D) and vpages.shape == kpages.shape
+    assert block_table.shape == (B, MP) and seqlens.shape == (B,)
+    out = np.empty((B, Hq, D), np.float64)
+    lse = np.empty((B, Hq), np.float64)
+    rc = _load().oracle_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table),
+                                     _ptr(seqlens), _ptr(sinks), B, NB, P, MP, Hq, Hkv, D,
+                                     int(window), float(scale), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode_paged: invalid sizes")
     return out, lse
 
 

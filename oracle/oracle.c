@@ -216,6 +216,72 @@ int oracle_decode(const uint16_t *q, const uint16_t *kc, const uint16_t *vc,
 }
 
 /*
+ * Single-token decode over a paged KV cache (page 4, "Dao-AILab/flash-attention"
+ * contributor guide: the module table's "Paged KV / decode" row and step 1 of
+ * its call walk-through, where the interface packs a block_table; page 1's
+ * sliding-window serving with W = 513).  The cache is a pool of NB physical
+ * pages of P positions, kp/vp [NB, P, Hkv, D] bf16 bits, and block_table
+ * [B, MP] int32 maps page number t / P of sequence b to its physical page:
+ * position t of sequence b is row t % P of page block_table[b * MP + t / P].
+ * An entry outside [0, NB) stands for a page whose rows are all zero.  With
+ * that cache, the result is oracle_decode's with Smax = MP * P: the query at
+ * position n-1 sees the keys [max(0, n-W), n-1] and the sink.
+ * out [B,Hq,D] f64, lse [B,Hq] f64 (may be NULL).
+ */
+int oracle_decode_paged(const uint16_t *q, const uint16_t *kp, const uint16_t *vp,
+                        const int32_t *block_table, const int32_t *seqlens,
+                        const float *sinks, int B, int NB, int P, int MP, int Hq,
+                        int Hkv, int D, int W, float scale, double *out,
+                        double *lse)
+{
+    if (B < 0 || NB < 0 || P <= 0 || MP < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 ||
+        W < 1 || Hq % Hkv)
+        return -1;
+    const int64_t smax = (int64_t)MP * P;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > smax) return -1;
+    const int group = Hq / Hkv;
+    const int64_t rows = (int64_t)B * Hq;
+#pragma omp parallel
+    {
+        /* the visible rows of one (sequence, kv head), gathered in order */
+        uint16_t *kr = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(smax > 0 ? smax : 1) * D);
+        uint16_t *vr = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(smax > 0 ? smax : 1) * D);
+        double *s = (double *)malloc(sizeof(double) * (size_t)(smax > 0 ? smax : 1));
+        double lse_row;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            int h = (int)(r % Hq);
+            int b = (int)(r / Hq);
+            int hk = h / group;
+            int n = seqlens[b];
+            int lo = n - W < 0 ? 0 : n - W;
+            for (int t = lo; t < n; ++t) {
+                int32_t page = block_table[(int64_t)b * MP + t / P];
+                int slot = t % P;
+                uint16_t *kd = kr + (int64_t)(t - lo) * D;
+                uint16_t *vd = vr + (int64_t)(t - lo) * D;
+                if (page < 0 || page >= NB) {
+                    memset(kd, 0, sizeof(uint16_t) * (size_t)D);
+                    memset(vd, 0, sizeof(uint16_t) * (size_t)D);
+                } else {
+                    int64_t off = (((int64_t)page * P + slot) * Hkv + hk) * D;
+                    memcpy(kd, kp + off, sizeof(uint16_t) * (size_t)D);
+                    memcpy(vd, vp + off, sizeof(uint16_t) * (size_t)D);
+                }
+            }
+            attend_row(q + r * D, kr, vr, D, 0, n - lo - 1, D, (double)scale,
+                       (double)sinks[h], s, out + r * D, &lse_row);
+            if (lse) lse[r] = lse_row;
+        }
+        free(s);
+        free(vr);
+        free(kr);
+    }
+    return 0;
+}
+
+/*
  * Split-KV step 1 (page 5, section 3): the partial softmax of one query row
  * over the keys [lo, hi] only, with no sink.  O_s is normalised within the
  * split and LSE_s is its natural-log normaliser.  Requires lo <= hi.
