@@ -138,6 +138,38 @@ int attn_sink_decode_chunked(const attn_tensor *q, const attn_tensor *kcache,
                              int32_t chunk, attn_tensor *out, void *stream);
 
 /*
+ * Single-token split-KV decode over a PAGED KV cache (page
+ * "Dao-AILab/flash-attention" contributor guide: module table row "Paged KV /
+ * decode" and step 1 of its call walk-through, where the interface packs a
+ * block_table; the window W of page "cf-1.com/news/6055759" applies as for
+ * attn_sink_decode).
+ *
+ *   q            [B, Hq, D]        bf16, as for attn_sink_decode.
+ *   kpages,
+ *   vpages       [NB, P, Hkv, D]   bf16 pools of NB physical pages of P
+ *                                  positions each; P a power of two in
+ *                                  [16, 65536].
+ *   block_table  [B, MP] int32, DEVICE memory (innermost stride 1): position
+ *                t of sequence b is row t % P of page block_table[b][t / P].
+ *                Pages may be shared between sequences.  An entry outside
+ *                [0, NB) reads as a page of zero rows (no fault).  Entries of
+ *                pages that hold no visible position may hold anything: they
+ *                are either not read or read and discarded.
+ *   seqlens      [B] int32, DEVICE memory, 0 <= n <= MP * P (clamped).
+ *   sinks, window, scale, out: as for attn_sink_decode (Smax = MP * P).
+ *
+ * The same three launches as attn_sink_decode; each 64-key tile is loaded
+ * from its page (P >= 64) or from 64/P pages (P = 16, 32) by TMA, so split
+ * ranges start at the 64-key boundary at or below the window's first key and
+ * the keys before the window are masked.  Workspace, supported D and Hq/Hkv:
+ * as for attn_sink_decode.
+ */
+int attn_sink_decode_paged(const attn_tensor *q, const attn_tensor *kpages,
+                           const attn_tensor *vpages, const attn_tensor *block_table,
+                           const attn_tensor *seqlens, const attn_tensor *sinks,
+                           int32_t window, float scale, attn_tensor *out, void *stream);
+
+/*
  * attn_sink_decode without any allocation (the pages have no counterpart to
  * this entry point; it is a deployment convenience).  Same arguments, result
  * and kernels as attn_sink_decode, but the split table and the partial

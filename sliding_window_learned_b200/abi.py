@@ -34,7 +34,8 @@ _DTYPES = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float32: ATTN_DTYPE_F32,
 
 # Every symbol include/attnsink.h declares.
 EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_cudacore", "attn_sink_decode",
-           "attn_sink_decode_chunked", "attn_sink_decode_noalloc", "attn_sink_get_status",
+           "attn_sink_decode_chunked", "attn_sink_decode_paged", "attn_sink_decode_noalloc",
+           "attn_sink_get_status",
            "attn_sink_strerror", "attn_sink_last_error")
 
 
@@ -71,6 +72,8 @@ def load() -> ctypes.CDLL:
         lib.attn_sink_decode.restype = ctypes.c_int
         lib.attn_sink_decode_chunked.argtypes = [P, P, P, P, P, i32, f32, i32, P, V]
         lib.attn_sink_decode_chunked.restype = ctypes.c_int
+        lib.attn_sink_decode_paged.argtypes = [P, P, P, P, P, P, i32, f32, P, V]
+        lib.attn_sink_decode_paged.restype = ctypes.c_int
         lib.attn_sink_decode_noalloc.argtypes = [P, P, P, P, P, i32, f32, P, V]
         lib.attn_sink_decode_noalloc.restype = ctypes.c_int
         lib.attn_sink_get_status.argtypes = [V]
@@ -169,6 +172,18 @@ def attn_sink_decode_chunked(q, kcache, vcache, seqlens, sinks, window: int, sca
                                       _ref(ds[4]), int(window), float(scale), int(chunk),
                                       _ref(ds[5]), _stream(stream, q))
     _check(rc, "attn_sink_decode_chunked")
+
+
+def attn_sink_decode_paged(q, kpages, vpages, block_table, seqlens, sinks, window: int,
+                           scale: float, out, stream=None):
+    """C ``attn_sink_decode_paged``: split-KV decode over page pools
+    ``[NB, P, Hkv, D]`` addressed through ``block_table [B, MP]`` (int32)."""
+    lib = load()
+    ds = [describe(x) for x in (q, kpages, vpages, block_table, seqlens, sinks, out)]
+    rc = lib.attn_sink_decode_paged(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]),
+                                    _ref(ds[4]), _ref(ds[5]), int(window), float(scale),
+                                    _ref(ds[6]), _stream(stream, q))
+    _check(rc, "attn_sink_decode_paged")
 
 
 def attn_sink_decode_noalloc(q, kcache, vcache, seqlens, sinks, window: int, scale: float, out,

@@ -351,6 +351,83 @@ int prep_decode(const attn_tensor *q, const attn_tensor *kcache, const attn_tens
   return ATTN_OK;
 }
 
+// Validates the paged-cache decode arguments and fills `out_args` (kc/vc are
+// the page pools, Smax = pages per sequence * page size); `*empty` as above.
+int prep_decode_paged(const attn_tensor *q, const attn_tensor *kpages, const attn_tensor *vpages,
+                      const attn_tensor *block_table, const attn_tensor *seqlens,
+                      const attn_tensor *sinks, int32_t window, float scale, attn_tensor *out,
+                      DecodeArgs *out_args, bool *empty) {
+  int rc;
+  *empty = false;
+  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 3, false))) return rc;
+  if ((rc = check_tensor(kpages, "kpages", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(vpages, "vpages", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(block_table, "block_table", ATTN_DTYPE_I32, 2, false))) return rc;
+  if ((rc = check_tensor(seqlens, "seqlens", ATTN_DTYPE_I32, 1, false))) return rc;
+  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(out, "out", ATTN_DTYPE_BF16, 3, false))) return rc;
+  const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t NB = kpages->shape[0], P = kpages->shape[1], Hkv = kpages->shape[2];
+  const int64_t MP = block_table->shape[1];
+  if (kpages->shape[3] != D) return fail(ATTN_EINVAL, "kpages head dim does not match q");
+  for (int d = 0; d < 4; ++d)
+    if (vpages->shape[d] != kpages->shape[d]) return fail(ATTN_EINVAL, "vpages shape does not match kpages");
+  for (int d = 0; d < 3; ++d)
+    if (out->shape[d] != q->shape[d]) return fail(ATTN_EINVAL, "out shape does not match q");
+  if (block_table->shape[0] != B) return fail(ATTN_EINVAL, "block_table must have B rows");
+  if (seqlens->shape[0] != B) return fail(ATTN_EINVAL, "seqlens must have B entries");
+  if (sinks->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks must have Hq entries");
+  if ((B > 1 && seqlens->stride[0] != 1) || (Hq > 1 && sinks->stride[0] != 1))
+    return fail(ATTN_EINVAL, "seqlens and sinks must be contiguous");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
+  if (P < 16 || P > 65536 || (P & (P - 1)))
+    return fail(ATTN_EUNSUPPORTED, "page size %lld must be a power of two in [16, 65536]", (long long)P);
+  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
+  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
+  if (D != 64 && D != 128 && D != 256) return fail(ATTN_EUNSUPPORTED, "head dim %lld not supported", (long long)D);
+  if (Hq / Hkv > (D == 256 ? 8 : 16)) return fail(ATTN_EUNSUPPORTED, "Hq/Hkv too large for this head dim");
+  if ((reinterpret_cast<uintptr_t>(q->data) % 4) || q->stride[0] % 2 || q->stride[1] % 2)
+    return fail(ATTN_EINVAL, "q rows must be 4-byte aligned");
+  if (B > (1 << 20) || NB > (1LL << 31) - 1 || MP * P > (1LL << 30))
+    return fail(ATTN_EUNSUPPORTED, "B, the pool or pages per sequence * page size too large");
+  if (B == 0 || Hq == 0) {
+    *empty = true;
+    return ATTN_OK;
+  }
+  DecodeArgs &a = *out_args;
+  a.q = q->data;
+  a.kc = kpages->data;
+  a.vc = vpages->data;
+  a.seqlens = static_cast<const int *>(seqlens->data);
+  a.sinks = static_cast<const float *>(sinks->data);
+  a.out = out->data;
+  a.B = static_cast<int>(B);
+  a.Smax = static_cast<int>(MP * P);
+  a.Hq = static_cast<int>(Hq);
+  a.Hkv = static_cast<int>(Hkv);
+  a.D = static_cast<int>(D);
+  a.W = window;
+  a.scale = scale;
+  // keep every sequence within 32 splits; the range may start 63 keys early
+  const int64_t vis = (window < a.Smax ? window : a.Smax) + 63;
+  int64_t c = ((vis + 31) / 32 + 63) / 64 * 64;
+  a.chunk = static_cast<int32_t>(c < 256 ? 256 : c);
+  for (int d = 0; d < 2; ++d) {
+    a.q_s[d] = q->stride[d];
+    a.o_s[d] = out->stride[d];
+  }
+  for (int d = 0; d < 3; ++d) {
+    a.kc_s[d] = kpages->stride[d];
+    a.vc_s[d] = vpages->stride[d];
+  }
+  a.block_table = static_cast<const int *>(block_table->data);
+  a.bt_s0 = block_table->stride[0];
+  a.page = static_cast<int>(P);
+  a.npages = static_cast<int>(NB);
+  a.max_pages = static_cast<int>(MP);
+  return ATTN_OK;
+}
+
 }  // namespace attnsink
 
 using namespace attnsink;
@@ -429,6 +506,31 @@ int attn_sink_decode(const attn_tensor *q, const attn_tensor *kcache, const attn
                      const attn_tensor *seqlens, const attn_tensor *sinks, int32_t window,
                      float scale, attn_tensor *out, void *stream) {
   return attn_sink_decode_chunked(q, kcache, vcache, seqlens, sinks, window, scale, 0, out, stream);
+}
+
+int attn_sink_decode_paged(const attn_tensor *q, const attn_tensor *kpages,
+                           const attn_tensor *vpages, const attn_tensor *block_table,
+                           const attn_tensor *seqlens, const attn_tensor *sinks, int32_t window,
+                           float scale, attn_tensor *out, void *stream) {
+  t_last_error[0] = '\0';
+  DecodeArgs a;
+  bool empty;
+  int rc = prep_decode_paged(q, kpages, vpages, block_table, seqlens, sinks, window, scale, out, &a,
+                             &empty);
+  if (rc || empty) return rc;
+  if ((rc = status_ptr(&a.status))) return rc;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  const size_t bytes = decode_workspace_bytes(a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void *ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, st);
+  if (e != cudaSuccess) return fail_cuda(e, "decode workspace allocation");
+  e = launch_decode(a, ws, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e != cudaSuccess) return fail_cuda(e, "attn_sink_decode_paged launch");
+  if (ef != cudaSuccess) return fail_cuda(ef, "decode workspace release");
+  return ATTN_OK;
 }
 
 int attn_sink_get_status(void *stream) {

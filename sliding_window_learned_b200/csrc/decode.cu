@@ -4,8 +4,14 @@
 //   plan     reads seqlens on the device; splits each sequence's visible key
 //            range [max(0, n-W), n) into chunks of `chunk` keys and lays the
 //            splits out contiguously (split_base[b] = exclusive prefix sum).
+//            For a paged cache the range first starts at the 64-key boundary
+//            below max(0, n-W), so that no key tile straddles two pages; the
+//            keys before the window are masked.
 //   split    persistent: one work item = (split, kv head).  A TMA producer
-//            warp streams 64-key K/V tiles of that head into a ring of stages;
+//            warp streams 64-key K/V tiles of that head into a ring of stages
+//            (for a paged cache, each tile from the pool page(s) the block
+//            table names: one box per tile, or 64/page boxes for pages of 16
+//            or 32 positions);
 //            four consumer warps each take 16 keys of every tile and run
 //            S^T = K q^T and O^T += V^T P^T on the warp-level tensor cores
 //            (the Hq/Hkv grouped query heads are the N = 8 dimension), with an
@@ -70,8 +76,8 @@ WsLayout ws_layout(const DecodeArgs &a) {
 
 // ------------------------------------------------------------------- plan
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int *seqlens, int B, int Smax,
-                                                           int W, int chunk, int *nsplit,
-                                                           int *base, int *ctrl) {
+                                                           int W, int chunk, int align,
+                                                           int *nsplit, int *base, int *ctrl) {
   __shared__ int warp_sums[32];
   const int t = threadIdx.x;
   const int per = (B + blockDim.x - 1) / blockDim.x;  // contiguous segment per thread
@@ -79,7 +85,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int *seqlens, i
   int local = 0;
   for (int b = b0; b < min(B, b0 + per); ++b) {
     const int n = min(max(seqlens[b], 0), Smax);
-    const int len = n - max(0, n - W);
+    const int len = n - max(0, n - W) / align * align;
     const int ns = (len + chunk - 1) / chunk;
     nsplit[b] = ns;
     local += ns;
@@ -127,11 +133,17 @@ struct SplitParams {
   int B, Smax, Hq, Hkv, G, W, chunk;
   float scale_log2;
   int *status;
+  // paged cache (page > 0): position t of sequence b is row t & (page - 1) of
+  // pool page block_table[b * bt_s0 + (t >> page_shift)]
+  const int *block_table;
+  int64_t bt_s0;
+  int page, page_shift, max_pages, align;
 };
 
 struct StageInfo {
   int b, hk, split, key0, nvalid, flags;  // flags: 1 first tile, 2 last tile, 4 end of work
-  int pad[2];
+  int nskip;                              // keys [0, nskip) of the tile precede the window
+  int pad;
 };
 
 template <int D, int NT>
@@ -209,10 +221,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = lo;
         const int split = g - p.base[b];
         const int n = min(max(p.seqlens[b], 0), p.Smax);
-        const int ks = max(0, n - p.W) + split * p.chunk;
+        const int vis0 = max(0, n - p.W);
+        const int ks = vis0 / p.align * p.align + split * p.chunk;
         const int ke = min(n, ks + p.chunk);
         const int nt = (ke - ks + kTK - 1) / kTK;
+        const int nbox = p.page == 0 ? 1 : kTK / min(kTK, p.page);   // boxes per tile (paged)
         for (int t = 0; ok && t < nt; ++t) {
+          // Paged cache: read the tile's page numbers before waiting for a free
+          // stage, so that the table reads overlap the wait.
+          int blk[4] = {0, 0, 0, 0};
+          if (p.page != 0) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              if (r >= nbox) break;
+              const int lp = (ks + t * kTK + r * (kTK / nbox)) >> p.page_shift;
+              blk[r] = lp < p.max_pages ? p.block_table[static_cast<int64_t>(b) * p.bt_s0 + lp] : -1;
+            }
+          }
           const int s = acquire();
           if (!ok) break;
           StageInfo &si = info[s];
@@ -221,12 +246,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           si.split = split;
           si.key0 = ks + t * kTK;
           si.nvalid = min(kTK, ke - si.key0);
+          si.nskip = max(0, vis0 - si.key0);
           si.flags = (t == 0 ? 1 : 0) | (t == nt - 1 ? 2 : 0);
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
           uint8_t *dst = smem + s * C::kStageBytes;
-          for (int c = 0; c < C::kChunks; ++c) {
-            tma_load_4d(dst + c * kTK * 128, &tmK, &full[s], c * 64, hk, si.key0, b);
-            tma_load_4d(dst + C::kTileBytes + c * kTK * 128, &tmV, &full[s], c * 64, hk, si.key0, b);
+          if (p.page == 0) {
+            for (int c = 0; c < C::kChunks; ++c) {
+              tma_load_4d(dst + c * kTK * 128, &tmK, &full[s], c * 64, hk, si.key0, b);
+              tma_load_4d(dst + C::kTileBytes + c * kTK * 128, &tmV, &full[s], c * 64, hk, si.key0, b);
+            }
+          } else {
+            // key0 is a multiple of 64 here, so each box of min(64, page) rows
+            // lies in one page.  A table entry outside the pool (or a page
+            // number past the table, for rows beyond the sequence end) loads
+            // zero rows: the box is out of range and filled, and it still
+            // delivers its bytes.
+            const int rows = kTK / nbox;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              if (r >= nbox) break;
+              const int r0 = r * rows;
+              const int slot = (si.key0 + r0) & (p.page - 1);
+              for (int c = 0; c < C::kChunks; ++c) {
+                tma_load_4d(dst + c * kTK * 128 + r0 * 128, &tmK, &full[s], c * 64, hk, slot, blk[r]);
+                tma_load_4d(dst + C::kTileBytes + c * kTK * 128 + r0 * 128, &tmV, &full[s], c * 64, hk,
+                            slot, blk[r]);
+              }
+            }
           }
         }
       }
@@ -287,12 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     const int key_w = warp * 16;  // this warp's 16 keys within the tile
-    // Keys past the end of the split are masked; where they are past the end
-    // of the sequence their cache rows may hold anything (NaN included), so
-    // their V rows are zeroed in shared memory before P.V reads them.
-    if (si.nvalid < key_w + 16) {
+    // Keys past the end of the split, and (paged cache) keys before the
+    // window, are masked; their cache rows may hold anything (NaN included),
+    // so their V rows are zeroed in shared memory before P.V reads them.
+    if (si.nvalid < key_w + 16 || si.nskip > key_w) {
       const int kidx = key_w + (lane & 15);
-      if (kidx >= si.nvalid) {
+      if (kidx >= si.nvalid || kidx < si.nskip) {
         for (int c = 0; c < C::kChunks; ++c) {
           uint8_t *row = smem + s * C::kStageBytes + C::kTileBytes + c * kTK * 128 + kidx * 128;
           const int half = lane >> 4;
@@ -322,7 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- online softmax per head (no sink here) ----
-    const bool v0 = key_w + g8 < si.nvalid, v1 = key_w + g8 + 8 < si.nvalid;
+    const int kv0 = key_w + g8, kv1 = key_w + g8 + 8;
+    const bool v0 = kv0 >= si.nskip && kv0 < si.nvalid, v1 = kv1 >= si.nskip && kv1 < si.nvalid;
     uint32_t pb[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -513,8 +560,14 @@ cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cu
   using C = DCfg<D, NT>;
   alignas(64) CUtensorMap mk, mv;
   cudaError_t e;
-  if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, kTK)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, kTK)) != cudaSuccess) return e;
+  if (a.page == 0) {
+    if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, kTK)) != cudaSuccess) return e;
+    if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, kTK)) != cudaSuccess) return e;
+  } else {
+    const int rows = a.page < kTK ? a.page : kTK;
+    if ((e = make_tma_bshd(&mk, a.kc, a.npages, a.page, a.Hkv, D, a.kc_s, rows)) != cudaSuccess) return e;
+    if ((e = make_tma_bshd(&mv, a.vc, a.npages, a.page, a.Hkv, D, a.vc_s, rows)) != cudaSuccess) return e;
+  }
   SplitParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
   p.q_sb = a.q_s[0];
@@ -535,6 +588,13 @@ cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cu
   p.chunk = a.chunk;
   p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.status = a.status;
+  p.block_table = a.block_table;
+  p.bt_s0 = a.bt_s0;
+  p.page = a.page;
+  p.page_shift = 0;
+  while (a.page > 0 && (1 << p.page_shift) < a.page) ++p.page_shift;
+  p.max_pages = a.max_pages;
+  p.align = a.page > 0 ? kTK : 1;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -563,7 +623,8 @@ cudaError_t launch_combine(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, 
 }  // namespace
 
 int decode_max_splits_per_seq(const DecodeArgs &a) {
-  const long long vis = a.W < a.Smax ? a.W : a.Smax;
+  // a paged cache's split range starts up to 63 keys before the window
+  const long long vis = (a.W < a.Smax ? a.W : a.Smax) + (a.page > 0 ? kTK - 1 : 0);
   return static_cast<int>((vis + a.chunk - 1) / a.chunk);
 }
 
@@ -573,6 +634,7 @@ cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t str
   const WsLayout w = ws_layout(a);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   decode_plan_kernel<<<1, 1024, 0, stream>>>(a.seqlens, a.B, a.Smax, a.W, a.chunk,
+                                             a.page > 0 ? kTK : 1,
                                              reinterpret_cast<int *>(ws + w.off_nsplit),
                                              reinterpret_cast<int *>(ws + w.off_base),
                                              reinterpret_cast<int *>(ws + w.off_ctrl));

@@ -22,7 +22,10 @@ struct FwdArgs {
 };
 
 // Decode: q/out [B,Hq,D], caches [B,Smax,Hkv,D] (bf16), seqlens [B] int32
-// (device), sinks [Hq] f32.
+// (device), sinks [Hq] f32.  With page > 0 the caches are page pools
+// [npages, page, Hkv, D] instead: position t of sequence b is row t % page of
+// pool page block_table[b * bt_s0 + t / page] (device int32), and
+// Smax = max_pages * page.
 struct DecodeArgs {
   const void *q, *kc, *vc;
   const int *seqlens;
@@ -33,6 +36,10 @@ struct DecodeArgs {
   int chunk;                               // keys per split (multiple of 64)
   int64_t q_s[2], kc_s[3], vc_s[3], o_s[2];
   int *status;
+  const int *block_table = nullptr;        // paged cache only
+  int64_t bt_s0 = 0;
+  int page = 0;                            // 0: contiguous cache; else a power of two >= 16
+  int npages = 0, max_pages = 0;
 };
 
 // Bytes of stream-ordered workspace one decode call needs (256-byte aligned

@@ -151,6 +151,37 @@ def test_decode_rejects_invalid_arguments(lib, case):
     assert rc == expect, (case, rc, abi.attn_sink_last_error())
 
 
+@pytest.mark.parametrize("case", ["page not a power of two", "page too small", "table rows",
+                                  "table dtype", "pool shapes differ", "gqa", "head dim"])
+def test_paged_decode_rejects_invalid_arguments(lib, case):
+    q, o = _t([2, 8, 128]), _t([2, 8, 128])
+    kp, vp = _t([40, 64, 2, 128]), _t([40, 64, 2, 128])
+    bt = _t([2, 16], abi.ATTN_DTYPE_I32)
+    sl, s = _t([2], abi.ATTN_DTYPE_I32), _t([8], abi.ATTN_DTYPE_F32)
+    expect = abi.ATTN_EINVAL
+    if case == "page not a power of two":
+        kp, vp = _t([40, 48, 2, 128]), _t([40, 48, 2, 128])
+        expect = abi.ATTN_EUNSUPPORTED
+    elif case == "page too small":
+        kp, vp = _t([40, 8, 2, 128]), _t([40, 8, 2, 128])
+        expect = abi.ATTN_EUNSUPPORTED
+    elif case == "table rows":
+        bt = _t([3, 16], abi.ATTN_DTYPE_I32)
+    elif case == "table dtype":
+        bt = _t([2, 16], abi.ATTN_DTYPE_F32)
+    elif case == "pool shapes differ":
+        vp = _t([41, 64, 2, 128])
+    elif case == "gqa":
+        kp, vp = _t([40, 64, 3, 128]), _t([40, 64, 3, 128])
+    elif case == "head dim":
+        q, o = _t([2, 8, 96]), _t([2, 8, 96])
+        kp, vp = _t([40, 64, 2, 96]), _t([40, 64, 2, 96])
+        expect = abi.ATTN_EUNSUPPORTED
+    r = ctypes.byref
+    rc = lib.attn_sink_decode_paged(r(q), r(kp), r(vp), r(bt), r(sl), r(s), 128, 0.125, r(o), None)
+    assert rc == expect, (case, rc, abi.attn_sink_last_error())
+
+
 def test_noalloc_decode_rejects_workspace_beyond_its_array(lib):
     """The no-allocation decode checks its workspace bound on the host and
     refuses, with a message naming both sizes, before any device work."""
