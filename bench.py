@@ -8,7 +8,10 @@ L2 (the prefill inputs are smaller than L2; the decode cache is ~17 GB).
 
 `value` is useful prefill TFLOP/s (window-visible pairs only), summed over
 ranks, from CUDA events around each prefill launch; the decode figure (HBM
-GB/s of algorithmic bytes) is reported beside it.  `--impl reference` times
+GB/s of algorithmic bytes) is reported beside it, and after the timed steps
+the same decode over a paged copy of its cache (256-position pages at random
+pool positions, attn_sink_decode_paged) is timed as `decode_paged`.
+`--impl reference` times
 the fp64 CPU oracle on a bounded sample of the same prefill workload.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -230,11 +233,41 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     t_e2e = e0.elapsed_time(e1) / 1e3
 
+    # ---- the same decode over a paged cache (256-position pages at random
+    # pool positions, addressed through a block table) ----
+    page = 256
+    n_pages = dcfg.B * (dcfg.Smax // page)
+    perm = torch.randperm(n_pages, generator=torch.Generator(device=dev).manual_seed(rank), device=dev)
+    kpool = torch.empty((n_pages, page, dcfg.Hkv, dcfg.D), dtype=torch.bfloat16, device=dev)
+    kpool[perm] = y["kcache"].reshape(n_pages, page, dcfg.Hkv, dcfg.D)
+    vpool = torch.empty_like(kpool)
+    vpool[perm] = y["vcache"].reshape(n_pages, page, dcfg.Hkv, dcfg.D)
+    table = perm.reshape(dcfg.B, dcfg.Smax // page).to(torch.int32)
+    del perm
+
+    def dec_paged():
+        swl.attn_sink_decode_paged(y["q"], kpool, vpool, table, y["seqlens"], y["sinks"], dcfg.W,
+                                   dcfg.scale, dout, stream)
+
+    Kp = max(3, min(K, 50))
+    for _ in range(3):
+        dec_paged()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Kp):
+        dec_paged()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if swl.attn_sink_get_status() != 0:
+        raise RuntimeError("device status error in the paged decode")
+    t_paged = e0.elapsed_time(e1) / 1e3
+    del kpool, vpool, table
+
     # ---- max over ranks ----
-    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e], dtype=torch.float64, device=dev)
+    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    t_fwd, t_dec, t_all, t_e2e = times.tolist()
+    t_fwd, t_dec, t_all, t_e2e, t_paged = times.tolist()
 
     if rank != 0:
         return
@@ -278,6 +311,11 @@ def run_ours(args, rank, world, local_rank):
                                 "traffic": profiled_traffic("decode_split", [
                                     "sliding_window_learned_b200/csrc/decode.cu",
                                     "sliding_window_learned_b200/csrc/ptx.cuh"])}},
+        "decode_paged": {"value": round(world * Kp * dbytes / t_paged / 1e9, 2), "unit": "GB/s",
+                         "page": page, "ms_per_call": round(t_paged / Kp * 1e3, 4),
+                         "frac": round(dbytes / (t_paged / Kp) / 1e9 / hbm_peak, 4),
+                         "what": "attn_sink_decode_paged on the decode workload, cache in 256-position "
+                                 "pages at random pool positions"},
         "e2e": {"value": round(world * Ke * fwd_flops / t_e2e / 1e12, 4), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "attn_sink_fwd with pinned host inputs copied in and O, LSE copied out each step"},
