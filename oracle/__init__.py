@@ -104,6 +104,32 @@ def fwd(q, k, v, sinks, window: int, scale: float, with_lse: bool = True):
     return out, lse
 
 
+def fwd_varlen(q, k, v, cu_seqlens, sinks, window: int, scale: float):
+    """Prefill forward over packed variable-length sequences: the tokens of
+    sequence b are rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of q [T,Hq,D] and
+    k/v [T,Hkv,D] (uint16 bf16 bits), and each sequence is attended on its own
+    (positions restart at 0; no query sees another sequence's keys), exactly
+    as one batch element of ``fwd`` (the varlen path of the flash-attention
+    contributor guide's call walk-through, step 2).
+    Returns (out [T,Hq,D] float64, lse [Hq,T] float64)."""
+    q, k, v, sinks = _u16(q), _u16(k), _u16(v), _f32(sinks)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    assert k.shape == (T, Hkv, D) and v.shape == k.shape
+    assert cu.ndim == 1 and cu[0] == 0 and cu[-1] == T and np.all(np.diff(cu) >= 0)
+    out = np.empty((T, Hq, D), np.float64)
+    lse = np.empty((Hq, T), np.float64)
+    for b in range(len(cu) - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        if s1 == s0:
+            continue
+        o_b, l_b = fwd(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], sinks, window, scale)
+        out[s0:s1] = o_b[0]
+        lse[:, s0:s1] = l_b[0]
+    return out, lse
+
+
 def fwd_rows(q, k, v, sinks, window: int, scale: float, rows):
     """The forward for selected rows only.  rows: int array [n, 3] of
     (b, i, h).  Returns (out [n, D] float64, lse [n] float64)."""
