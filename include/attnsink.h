@@ -87,6 +87,33 @@ int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
                   attn_tensor *out, attn_tensor *lse, void *stream);
 
 /*
+ * Prefill forward over packed variable-length sequences (the varlen path of
+ * page "Dao-AILab/flash-attention" contributor guide, call walk-through step
+ * 2: cu_seqlens turned into per-sequence query tiles), with the learned sink
+ * and window of attn_sink_fwd.  Each sequence is attended on its own: its
+ * positions restart at 0 and no query sees another sequence's keys.
+ *
+ *   q           [T, Hq, D]  bf16, the sequences' rows one after another
+ *   k, v        [T, Hkv, D] bf16
+ *   cu_seqlens  [B + 1] int32, DEVICE memory: sequence b is rows
+ *               cu_seqlens[b] .. cu_seqlens[b+1]-1; cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[B] = T (empty sequences allowed).
+ *               Values are clamped to [0, T] on the device, so a malformed
+ *               table gives wrong rows but no access outside the tensors.
+ *   max_seqlen  host int >= every sequence's length (sizes the work grid;
+ *               rows of a longer sequence past max_seqlen are not written).
+ *   sinks, window, scale: as for attn_sink_fwd.
+ *   out         [T, Hq, D]  bf16.
+ *   lse         [Hq, T]     f32 or NULL (innermost stride 1).
+ * Supported head dims D: 64, 128, 256.  B = 0, T = 0 or max_seqlen = 0 is a
+ * no-op.  Runs on the tcgen05/TMEM tensor-core kernel of attn_sink_fwd.
+ */
+int attn_sink_fwd_varlen(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                         const attn_tensor *cu_seqlens, int32_t max_seqlen,
+                         const attn_tensor *sinks, int32_t window, float scale,
+                         attn_tensor *out, attn_tensor *lse, void *stream);
+
+/*
  * The same operation on a plain CUDA-core fp32 kernel (one warp per output
  * row).  Slow; it is an independent second implementation for verification
  * and debugging, with the same arguments and semantics as attn_sink_fwd, and

@@ -33,7 +33,7 @@ _DTYPES = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float32: ATTN_DTYPE_F32,
            torch.int32: ATTN_DTYPE_I32}
 
 # Every symbol include/attnsink.h declares.
-EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_cudacore", "attn_sink_decode",
+EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_varlen", "attn_sink_fwd_cudacore", "attn_sink_decode",
            "attn_sink_decode_chunked", "attn_sink_decode_paged", "attn_sink_decode_noalloc",
            "attn_sink_get_status",
            "attn_sink_strerror", "attn_sink_last_error")
@@ -68,6 +68,8 @@ def load() -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.argtypes = [P, P, P, P, i32, f32, P, P, V]
             fn.restype = ctypes.c_int
+        lib.attn_sink_fwd_varlen.argtypes = [P, P, P, P, i32, P, i32, f32, P, P, V]
+        lib.attn_sink_fwd_varlen.restype = ctypes.c_int
         lib.attn_sink_decode.argtypes = [P, P, P, P, P, i32, f32, P, V]
         lib.attn_sink_decode.restype = ctypes.c_int
         lib.attn_sink_decode_chunked.argtypes = [P, P, P, P, P, i32, f32, i32, P, V]
@@ -141,6 +143,18 @@ def attn_sink_fwd(q, k, v, sinks, window: int, scale: float, out, lse=None, stre
     rc = lib.attn_sink_fwd(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), int(window),
                            float(scale), _ref(ds[4]), _ref(ds[5]), _stream(stream, q))
     _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, sinks, window: int, scale: float,
+                         out, lse=None, stream=None):
+    """C ``attn_sink_fwd_varlen``: forward over packed sequences (q/out
+    [T,Hq,D], k/v [T,Hkv,D], cu_seqlens [B+1] int32 on the device, lse [Hq,T])."""
+    lib = load()
+    ds = [describe(x) for x in (q, k, v, cu_seqlens, sinks, out, lse)]
+    rc = lib.attn_sink_fwd_varlen(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]),
+                                  int(max_seqlen), _ref(ds[4]), int(window), float(scale),
+                                  _ref(ds[5]), _ref(ds[6]), _stream(stream, q))
+    _check(rc, "attn_sink_fwd_varlen")
 
 
 def attn_sink_fwd_cudacore(q, k, v, sinks, window: int, scale: float, out, lse=None, stream=None):

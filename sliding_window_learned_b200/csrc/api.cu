@@ -186,6 +186,67 @@ int prep_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
   return ATTN_OK;
 }
 
+// Validates the packed variable-length forward's arguments and fills `a`.
+int prep_fwd_varlen(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                    const attn_tensor *cu_seqlens, int32_t max_seqlen, const attn_tensor *sinks,
+                    int32_t window, float scale, attn_tensor *out, attn_tensor *lse, FwdArgs *a) {
+  int rc;
+  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 3, true))) return rc;
+  if ((rc = check_tensor(k, "k", ATTN_DTYPE_BF16, 3, true))) return rc;
+  if ((rc = check_tensor(v, "v", ATTN_DTYPE_BF16, 3, true))) return rc;
+  if ((rc = check_tensor(cu_seqlens, "cu_seqlens", ATTN_DTYPE_I32, 1, false))) return rc;
+  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(out, "out", ATTN_DTYPE_BF16, 3, true))) return rc;
+  const int64_t T = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+  const int64_t Hkv = k->shape[1];
+  if (k->shape[0] != T || k->shape[2] != D) return fail(ATTN_EINVAL, "k shape does not match q");
+  for (int d = 0; d < 3; ++d) {
+    if (v->shape[d] != k->shape[d]) return fail(ATTN_EINVAL, "v shape does not match k");
+    if (out->shape[d] != q->shape[d]) return fail(ATTN_EINVAL, "out shape does not match q");
+  }
+  if (cu_seqlens->shape[0] < 1) return fail(ATTN_EINVAL, "cu_seqlens needs B + 1 >= 1 entries");
+  if (cu_seqlens->shape[0] > 1 && cu_seqlens->stride[0] != 1) return fail(ATTN_EINVAL, "cu_seqlens must be contiguous");
+  if (sinks->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks must have Hq = %lld entries", (long long)Hq);
+  if (sinks->shape[0] > 1 && sinks->stride[0] != 1) return fail(ATTN_EINVAL, "sinks must be contiguous");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
+  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
+  if (max_seqlen < 0) return fail(ATTN_EINVAL, "max_seqlen must be >= 0");
+  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
+  if (lse) {
+    if ((rc = check_tensor(lse, "lse", ATTN_DTYPE_F32, 2, false))) return rc;
+    if (lse->shape[0] != Hq || lse->shape[1] != T) return fail(ATTN_EINVAL, "lse must be [Hq, T]");
+  }
+  const int64_t B = cu_seqlens->shape[0] - 1;
+  if (B > 65535 || Hq > 65535 || T > (1LL << 30))
+    return fail(ATTN_EUNSUPPORTED, "B and Hq must be <= 65535 and T <= 2^30");
+  a->q = q->data;
+  a->k = k->data;
+  a->v = v->data;
+  a->sinks = static_cast<const float *>(sinks->data);
+  a->out = out->data;
+  a->lse = lse ? static_cast<float *>(lse->data) : nullptr;
+  a->B = static_cast<int>(B);
+  a->L = max_seqlen;
+  a->T = static_cast<int>(T);
+  a->Hq = static_cast<int>(Hq);
+  a->Hkv = static_cast<int>(Hkv);
+  a->D = static_cast<int>(D);
+  a->W = window;
+  a->scale = scale;
+  a->cu_seqlens = static_cast<const int *>(cu_seqlens->data);
+  // one batch slice of T rows: its (unused) batch stride spans the slice
+  const attn_tensor *ts[4] = {q, k, v, out};
+  int64_t *ss[4] = {a->q_s, a->k_s, a->v_s, a->o_s};
+  for (int x = 0; x < 4; ++x) {
+    ss[x][0] = (T > 0 ? T : 1) * ts[x]->stride[0];
+    ss[x][1] = ts[x]->stride[0];
+    ss[x][2] = ts[x]->stride[1];
+  }
+  a->lse_s[0] = 0;
+  a->lse_s[1] = lse ? lse->stride[0] : 0;
+  return ATTN_OK;
+}
+
 }  // namespace
 
 // TMA descriptor for a [d3, d2, d1, d0] bf16 tensor, box {64, 1, box_rows, 1},
@@ -461,6 +522,22 @@ int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
   if ((rc = status_ptr(&a.status))) return rc;
   const cudaError_t e = launch_fwd_tc(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd launch");
+}
+
+int attn_sink_fwd_varlen(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                         const attn_tensor *cu_seqlens, int32_t max_seqlen,
+                         const attn_tensor *sinks, int32_t window, float scale, attn_tensor *out,
+                         attn_tensor *lse, void *stream) {
+  t_last_error[0] = '\0';
+  FwdArgs a;
+  int rc = prep_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, sinks, window, scale, out, lse, &a);
+  if (rc) return rc;
+  if (a.D != 64 && a.D != 128 && a.D != 256)
+    return fail(ATTN_EUNSUPPORTED, "head dim %d not supported (64, 128, 256)", a.D);
+  if (a.B == 0 || a.T == 0 || a.L == 0) return ATTN_OK;
+  if ((rc = status_ptr(&a.status))) return rc;
+  const cudaError_t e = launch_fwd_tc(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd_varlen launch");
 }
 
 int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,

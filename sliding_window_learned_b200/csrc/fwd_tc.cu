@@ -117,6 +117,13 @@ struct Params {
   float *lse;
   int64_t lse_sb, lse_sh;
   int *status;
+  // Packed variable-length sequences (null: a [B, L] batch).  Sequence b is
+  // rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of [T, H, D] tensors; the last,
+  // ragged query tile of a sequence is stored row by row through `out`.
+  const int *cu_seqlens;
+  int T;
+  __nv_bfloat16 *out;
+  int64_t o_sr, o_sh;
 };
 
 // Warp-uniform bounded wait: every lane learns the same outcome, so the
@@ -347,7 +354,9 @@ __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col,
   return true;
 }
 
-template <int D, int BN, int NH>
+// kPacked: packed variable-length sequences (Params::cu_seqlens); a separate
+// instantiation, so that the batched kernel carries none of its code.
+template <int D, int BN, int NH, bool kPacked>
 __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -379,9 +388,15 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   // see the most keys under a causal window), head groups fastest so that the
   // CTAs running at the same time share K/V tiles in L2.  CTA c takes units
   // c, c + gridDim.x, ...
+  // A unit's sequence has `len` positions starting at row `row0` of the
+  // row dimension, in batch slice bc() of the tensor maps; with packed
+  // sequences a unit past its sequence's end is empty (n_tiles = 0) and every
+  // role skips it.
   struct Unit {
-    int m0, h0, b, kt0, n_tiles;
+    int m0, h0, b, kt0, n_tiles, len, row0;
   };
+  constexpr bool packed = kPacked;
+  auto bc = [&](const Unit &t) { return packed ? 0 : t.b; };
   auto unit_at = [&](int u) {
     Unit t;
     const int per_m = HP * p.B;
@@ -390,9 +405,18 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
     t.h0 = (r % HP) * NH;
     t.b = r / HP;
     t.m0 = mt * kBM;
-    const int row_last = min(p.L - 1, t.m0 + kBM - 1);
+    if constexpr (packed) {
+      // offsets clamped to [0, T], so that a malformed table never moves a
+      // store outside the tensors
+      t.row0 = min(max(p.cu_seqlens[t.b], 0), p.T);
+      t.len = min(max(p.cu_seqlens[t.b + 1], t.row0), p.T) - t.row0;
+    } else {
+      t.row0 = 0;
+      t.len = p.L;
+    }
+    const int row_last = min(t.len - 1, t.m0 + kBM - 1);
     t.kt0 = max(0, t.m0 - p.W + 1) / BN;
-    t.n_tiles = row_last / BN - t.kt0 + 1;
+    t.n_tiles = t.m0 < t.len ? row_last / BN - t.kt0 + 1 : 0;
     return t;
   };
 
@@ -460,8 +484,11 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
           tma_load_4d(dst + c * BN * 128, map, &full[s], c * 64, 0, kt * BN, b);
         ++slot;
       };
-      for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; ++ul, u += gridDim.x) {
+      int ul = -1;                            // units that are not empty, so far
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const Unit t = unit_at(u);
+        if (packed && t.n_tiles <= 0) continue;
+        ++ul;
         const int qb = ul & 1;
         // the buffer's previous unit has stored its O out of it
         if (ul >= 2 &&
@@ -473,7 +500,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         for (int w = 0; w < NH; ++w)
           for (int c = 0; c < C::kChunks; ++c)
             tma_load_4d(sQ + qb * C::kQBufBytes + w * C::kQTileBytes + c * kBM * 128, &tmQ,
-                        &q_full[qb], c * 64, t.h0 + w, t.m0, t.b);
+                        &q_full[qb], c * 64, t.h0 + w, t.row0 + t.m0, bc(t));
         q_loaded = ul + 1;
         const int hk = t.h0 / p.group;
         // the order the MMA warp consumes: K_0 .. K_{kSBuf-1}, then per tile
@@ -488,7 +515,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
           mbar_arrive_expect_tx(&full[s], C::kTileBytes);
           uint8_t *dst = sRing + s * C::kTileBytes;
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_4d(dst + c * BN * 128, map, &full[s], c * 64, hk, kt * BN, t.b);
+            tma_load_4d(dst + c * BN * 128, map, &full[s], c * 64, hk, t.row0 + kt * BN, bc(t));
           ++slot;
         };
         for (int jj = 0; ok && jj < C::kSBuf && jj < t.n_tiles; ++jj) kv(&tmK, t.kt0 + jj);
@@ -531,8 +558,9 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         return ok;
       };
       int jg = 0;                            // tiles of earlier units (barrier phases)
-      for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; ++ul, u += gridDim.x) {
+      for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const Unit t = unit_at(u);
+        if (packed && t.n_tiles <= 0) continue;   // ul counts the units that are not empty
         const int qb = ul & 1;
         if (!mbar_wait(&q_full[qb], static_cast<uint32_t>(ul >> 1) & 1u, ctx, kWhereQ)) {
           ok = false;
@@ -604,6 +632,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         }
         jg += t.n_tiles;
         umma_commit(o_full);                 // this unit's O is complete
+        ++ul;
       }
       // Every tensor-core operation of this CTA has finished before teardown.
       umma_commit(mma_done);
@@ -627,8 +656,11 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
     bool ok = true;
     int jg = 0;
     int pending_qb = -1;                             // buffer whose O store may still read it
-    for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; ++ul, u += gridDim.x) {
+    int ul = -1;                                     // units that are not empty, so far
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
       const Unit t = unit_at(u);
+      if (packed && t.n_tiles <= 0) continue;
+      ++ul;
       const int qb = ul & 1;
       const int h = t.h0 + w;
       const int i = t.m0 + r;                        // query position
@@ -646,9 +678,9 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         const int kbase = (t.kt0 + j) * BN;
         // Tile-uniform test: does any (row, key) of this tile fall outside the
         // causal window or past the end of the sequence?
-        const bool edge = (kbase + BN - 1 > t.m0) || (kbase < t.m0 + kBM - p.W) || (kbase + BN > p.L);
+        const bool edge = (kbase + BN - 1 > t.m0) || (kbase < t.m0 + kBM - p.W) || (kbase + BN > t.len);
         const int lo = i - p.W + 1 - kbase;          // first visible column
-        const int hi = min(i, p.L - 1) - kbase;      // last visible column
+        const int hi = min(i, t.len - 1) - kbase;    // last visible column
         // Per 32-column chunk, a warp-uniform class: every lane's visible
         // interval [lo, hi] covers the chunk (no mask), misses it (no work:
         // P = 0), or cuts it (per-element mask).
@@ -693,10 +725,13 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       const float lse_val = (l2 > 0.f) ? (new_m + log2f(l2)) * kLn2 : -INFINITY;
 
       // O^w (fp32, TMEM) -> bf16 -> swizzled staging tile (this unit's Q^w
-      // buffer, no longer read) -> TMA store; rows past the end of the
-      // sequence are clipped.  Once O^w is out of TMEM the next unit's PV^w
-      // may overwrite it.
+      // buffer, no longer read) -> TMA store; rows past the end of a batch
+      // tensor are clipped by the store.  The ragged last tile of a packed
+      // sequence is instead written row by row from registers (rows past the
+      // sequence's end belong to the next sequence).  Once O^w is out of TMEM
+      // the next unit's PV^w may overwrite it.
       uint8_t *stage = sQ + qb * C::kQBufBytes + w * C::kQTileBytes;
+      const bool direct = packed && t.m0 + kBM > t.len;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -710,8 +745,14 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
           v.y = pack_bf16x2(__uint_as_float(o[8 * uu + 2]) * oscale, __uint_as_float(o[8 * uu + 3]) * oscale);
           v.z = pack_bf16x2(__uint_as_float(o[8 * uu + 4]) * oscale, __uint_as_float(o[8 * uu + 5]) * oscale);
           v.w = pack_bf16x2(__uint_as_float(o[8 * uu + 6]) * oscale, __uint_as_float(o[8 * uu + 7]) * oscale);
-          const int unit = (c & 1) * 4 + uu;        // 16-byte unit within the 128-byte row
-          *reinterpret_cast<uint4 *>(chunk + ((unit ^ (r & 7)) << 4)) = v;
+          if (direct) {
+            if (i < t.len)
+              *reinterpret_cast<uint4 *>(p.out + static_cast<int64_t>(t.row0 + i) * p.o_sr +
+                                         static_cast<int64_t>(h) * p.o_sh + c * 32 + uu * 8) = v;
+          } else {
+            const int unit = (c & 1) * 4 + uu;      // 16-byte unit within the 128-byte row
+            *reinterpret_cast<uint4 *>(chunk + ((unit ^ (r & 7)) << 4)) = v;
+          }
         }
       }
       tc_fence_before();
@@ -722,12 +763,16 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       else
         named_barrier_sync(kBarEpilogue0 + 1, 128);
       if (r == 0) {
-        for (int c = 0; c < C::kChunks; ++c) tma_store_4d(&tmO, stage + c * kBM * 128, c * 64, h, t.m0, t.b);
-        tma_store_commit();
-        pending_qb = qb;
+        if (!direct) {
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_store_4d(&tmO, stage + c * kBM * 128, c * 64, h, t.row0 + t.m0, bc(t));
+          tma_store_commit();
+        }
+        pending_qb = qb;                           // released at the next unit's first tile
       }
-      if (p.lse != nullptr && i < p.L)
-        p.lse[static_cast<int64_t>(t.b) * p.lse_sb + static_cast<int64_t>(h) * p.lse_sh + i] = lse_val;
+      if (p.lse != nullptr && i < t.len)
+        p.lse[(packed ? t.row0 : static_cast<int64_t>(t.b) * p.lse_sb) + static_cast<int64_t>(h) * p.lse_sh +
+              i] = lse_val;
     }
     // stores must have read shared memory before the CTA leaves
     if (r == 0) tma_store_wait_all();
@@ -737,15 +782,18 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   }
 }
 
-template <int D, int BN, int NH>
+template <int D, int BN, int NH, bool kPacked>
 cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
   using C = Cfg<D, BN, NH>;
   alignas(64) CUtensorMap mq, mk, mv, mo;
   cudaError_t e;
-  if ((e = make_tma_bshd(&mq, a.q, a.B, a.L, a.Hq, D, a.q_s, kBM)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mk, a.k, a.B, a.L, a.Hkv, D, a.k_s, BN)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mv, a.v, a.B, a.L, a.Hkv, D, a.v_s, BN)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mo, a.out, a.B, a.L, a.Hq, D, a.o_s, kBM)) != cudaSuccess) return e;
+  // packed sequences: one [T, H, D] slice; else the [B, L, H, D] batch
+  const int64_t nb = a.cu_seqlens != nullptr ? 1 : a.B;
+  const int64_t nrow = a.cu_seqlens != nullptr ? a.T : a.L;
+  if ((e = make_tma_bshd(&mq, a.q, nb, nrow, a.Hq, D, a.q_s, kBM)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mk, a.k, nb, nrow, a.Hkv, D, a.k_s, BN)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mv, a.v, nb, nrow, a.Hkv, D, a.v_s, BN)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mo, a.out, nb, nrow, a.Hq, D, a.o_s, kBM)) != cudaSuccess) return e;
   Params p;
   p.L = a.L;
   p.Hq = a.Hq;
@@ -760,8 +808,13 @@ cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
   p.lse_sb = a.lse_s[0];
   p.lse_sh = a.lse_s[1];
   p.status = a.status;
-  auto kern = fwd_tc_kernel<D, BN, NH>;
-  static bool attr_set[64] = {};  // once per device
+  p.cu_seqlens = a.cu_seqlens;
+  p.T = a.T;
+  p.out = static_cast<__nv_bfloat16 *>(a.out);
+  p.o_sr = a.o_s[1];
+  p.o_sh = a.o_s[2];
+  auto kern = fwd_tc_kernel<D, BN, NH, kPacked>;
+  static bool attr_set[64] = {};  // once per device (per instantiation)
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
@@ -787,10 +840,16 @@ cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream) {
   // Two query heads per CTA when they share a kv head (even group size) and
   // their S and O fit TMEM together; otherwise one.
   const bool pair = (a.Hq / a.Hkv) % 2 == 0;
+  const bool packed = a.cu_seqlens != nullptr;
   switch (a.D) {
-    case 64: return pair ? launch<64, 128, 2>(a, stream) : launch<64, 64, 1>(a, stream);
-    case 128: return pair ? launch<128, 128, 2>(a, stream) : launch<128, 64, 1>(a, stream);
-    case 256: return launch<256, 64, 1>(a, stream);
+    case 64:
+      if (packed) return pair ? launch<64, 128, 2, true>(a, stream) : launch<64, 64, 1, true>(a, stream);
+      return pair ? launch<64, 128, 2, false>(a, stream) : launch<64, 64, 1, false>(a, stream);
+    case 128:
+      if (packed) return pair ? launch<128, 128, 2, true>(a, stream) : launch<128, 64, 1, true>(a, stream);
+      return pair ? launch<128, 128, 2, false>(a, stream) : launch<128, 64, 1, false>(a, stream);
+    case 256:
+      return packed ? launch<256, 64, 1, true>(a, stream) : launch<256, 64, 1, false>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }

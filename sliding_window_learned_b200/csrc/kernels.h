@@ -19,6 +19,13 @@ struct FwdArgs {
   int64_t q_s[3], k_s[3], v_s[3], o_s[3];  // strides of dims 0..2
   int64_t lse_s[2];                        // strides of dims 0..1
   int *status;                             // device status word (2 ints)
+  // Packed variable-length sequences: q/out [T,Hq,D], k/v [T,Hkv,D] viewed as
+  // one batch slice (strides of dim 0 = T * row stride), sequence b is rows
+  // cu_seqlens[b] .. cu_seqlens[b+1]-1 (device int32), B = number of
+  // sequences, L = an upper bound on their lengths, lse [Hq, T] (lse_s[1] =
+  // head stride).  Null: the [B, L] batch above.
+  const int *cu_seqlens = nullptr;
+  int T = 0;
 };
 
 // Decode: q/out [B,Hq,D], caches [B,Smax,Hkv,D] (bf16), seqlens [B] int32
