@@ -10,7 +10,9 @@ L2 (the prefill inputs are smaller than L2; the decode cache is ~17 GB).
 ranks, from CUDA events around each prefill launch; the decode figure (HBM
 GB/s of algorithmic bytes) is reported beside it, and after the timed steps
 the same decode over a paged copy of its cache (256-position pages at random
-pool positions, attn_sink_decode_paged) is timed as `decode_paged`.
+pool positions, attn_sink_decode_paged) is timed as `decode_paged`, and the
+forward over a seeded mix of 24 packed sequences (attn_sink_fwd_varlen) as
+`fwd_varlen`.
 `--impl reference` times
 the fp64 CPU oracle on a bounded sample of the same prefill workload.
 
@@ -263,11 +265,46 @@ def run_ours(args, rank, world, local_rank):
     t_paged = e0.elapsed_time(e1) / 1e3
     del kpool, vpool, table
 
+    # ---- the forward over packed variable-length sequences: a seeded mix of
+    # 24 sequences of U[1, 4096] tokens at the prefill workload's heads ----
+    vl_rng = np.random.default_rng(1000 + rank)
+    vl_lens = [int(n) for n in vl_rng.integers(1, 4097, size=24)]
+    vl_T = sum(vl_lens)
+    vl_gen = torch.Generator(device=dev).manual_seed(rank)
+    vq = torch.randn(vl_T, pcfg.Hq, pcfg.D, device=dev, generator=vl_gen).bfloat16()
+    vk = torch.randn(vl_T, pcfg.Hkv, pcfg.D, device=dev, generator=vl_gen).bfloat16()
+    vv = torch.randn(vl_T, pcfg.Hkv, pcfg.D, device=dev, generator=vl_gen).bfloat16()
+    vcu = torch.tensor(np.concatenate([[0], np.cumsum(vl_lens)]), dtype=torch.int32, device=dev)
+    vout = torch.empty_like(vq)
+    vlse = torch.empty(pcfg.Hq, vl_T, dtype=torch.float32, device=dev)
+    vl_flops = sum(4.0 * pcfg.D * pcfg.Hq * float(np.minimum(np.arange(n) + 1, pcfg.W).sum())
+                   for n in vl_lens)
+
+    def fwd_varlen():
+        swl.attn_sink_fwd_varlen(vq, vk, vv, vcu, max(vl_lens), sinks, pcfg.W, pcfg.scale, vout, vlse,
+                                 stream)
+
+    Kv = max(3, min(K, 50))
+    for _ in range(3):
+        fwd_varlen()
+    torch.cuda.synchronize()
+    t_varlen = 0.0
+    for _ in range(Kv):
+        flush.fill_(1.0)
+        e0.record(stream)
+        fwd_varlen()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_varlen += e0.elapsed_time(e1) / 1e3
+    if swl.attn_sink_get_status() != 0:
+        raise RuntimeError("device status error in the packed forward")
+    del vq, vk, vv, vout, vlse
+
     # ---- max over ranks ----
-    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged], dtype=torch.float64, device=dev)
+    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    t_fwd, t_dec, t_all, t_e2e, t_paged = times.tolist()
+    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen = times.tolist()
 
     if rank != 0:
         return
@@ -316,6 +353,11 @@ def run_ours(args, rank, world, local_rank):
                          "frac": round(dbytes / (t_paged / Kp) / 1e9 / hbm_peak, 4),
                          "what": "attn_sink_decode_paged on the decode workload, cache in 256-position "
                                  "pages at random pool positions"},
+        "fwd_varlen": {"value": round(world * Kv * vl_flops / t_varlen / 1e12, 3), "unit": "TFLOP/s",
+                       "ms_per_call": round(t_varlen / Kv * 1e3, 5),
+                       "frac": round(vl_flops / (t_varlen / Kv) / 1e12 / bf16_peak, 4),
+                       "what": "attn_sink_fwd_varlen on 24 packed sequences of U[1, 4096] tokens "
+                               f"(T = {vl_T}), Hq32 Hkv4 D128 W513, L2 flushed before each call"},
         "e2e": {"value": round(world * Ke * fwd_flops / t_e2e / 1e12, 4), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "attn_sink_fwd with pinned host inputs copied in and O, LSE copied out each step"},
