@@ -57,6 +57,10 @@ def _load():
         lib.oracle_decode.restype = I
         lib.oracle_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P]
         lib.oracle_decode_paged.restype = I
+        lib.oracle_decode_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P]
+        lib.oracle_decode_fp8.restype = I
+        lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f64.restype = ctypes.c_double
         lib.oracle_split_partial.argtypes = [P, P, P, ctypes.c_int64, I, I, I, F, P, P]
         lib.oracle_split_partial.restype = I
         lib.oracle_combine.argtypes = [I, P, P, I, F, P, P]
@@ -191,6 +195,38 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, sinks, window: int, sc
                                      int(window), float(scale), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_decode_paged: invalid sizes")
+    return out, lse
+
+
+def e4m3_to_f64(code: int) -> float:
+    """The oracle's FP8 e4m3 decoder (see oracle.c) for one byte."""
+    return float(_load().oracle_e4m3_to_f64(int(code) & 0xFF))
+
+
+def decode_fp8(q, kcache, vcache, k_descale, v_descale, seqlens, sinks, window: int,
+               scale: float):
+    """Single-token decode over an FP8 e4m3 KV cache (see oracle.c).
+
+    q [B,Hq,D] uint16 bf16 bits; kcache/vcache [B,Smax,Hkv,D] uint8 e4m3
+    codes; k_descale/v_descale [Hkv] float32 (key row = k_descale[hk] *
+    e4m3(row), value row likewise); seqlens [B] int32; sinks [Hq] float32.
+    Returns (out [B,Hq,D], lse [B,Hq]) float64."""
+    q, sinks = _u16(q), _f32(sinks)
+    kcache = np.ascontiguousarray(kcache, dtype=np.uint8)
+    vcache = np.ascontiguousarray(vcache, dtype=np.uint8)
+    k_descale, v_descale = _f32(k_descale), _f32(v_descale)
+    seqlens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    B, Hq, D = q.shape
+    _, Smax, Hkv, _ = kcache.shape
+    assert kcache.shape == (B, Smax, Hkv, D) and vcache.shape == kcache.shape
+    assert k_descale.shape == (Hkv,) and v_descale.shape == (Hkv,)
+    out = np.empty((B, Hq, D), np.float64)
+    lse = np.empty((B, Hq), np.float64)
+    rc = _load().oracle_decode_fp8(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(k_descale),
+                                   _ptr(v_descale), _ptr(seqlens), _ptr(sinks), B, Smax, Hq,
+                                   Hkv, D, int(window), float(scale), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_decode_fp8: invalid sizes")
     return out, lse
 
 

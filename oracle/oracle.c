@@ -282,6 +282,85 @@ int oracle_decode_paged(const uint16_t *q, const uint16_t *kp, const uint16_t *v
 }
 
 /*
+ * FP8 e4m3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent
+ * 0 is subnormal, m * 2^-9; S.1111.111 is NaN; no infinities) to double,
+ * written from that definition.
+ */
+static double e4m3_to_f64(uint8_t b)
+{
+    int sign = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+double oracle_e4m3_to_f64(uint8_t b) { return e4m3_to_f64(b); }
+
+/*
+ * Single-token decode over an FP8 (e4m3) KV cache with one dequantisation
+ * scale per kv head: the key row is k_descale[hk] * e4m3(kc row) and the value
+ * row v_descale[hk] * e4m3(vc row).  Page 1, "fix 2", applies v_descale to the
+ * output scale (rcp(row_sum) * sink_rescale * v_descale); its FP8 max_offset
+ * belongs to an FP8 P, and P is not quantised here, so it is 0.  Otherwise as
+ * oracle_decode: kc/vc [B,Smax,Hkv,D] bytes, out [B,Hq,D], lse [B,Hq].
+ */
+int oracle_decode_fp8(const uint16_t *q, const uint8_t *kc, const uint8_t *vc,
+                      const float *k_descale, const float *v_descale,
+                      const int32_t *seqlens, const float *sinks, int B, int Smax,
+                      int Hq, int Hkv, int D, int W, float scale, double *out,
+                      double *lse)
+{
+    if (B < 0 || Smax < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || W < 1 || Hq % Hkv)
+        return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Smax) return -1;
+    const int group = Hq / Hkv;
+    const int64_t rows = (int64_t)B * Hq;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Smax > 0 ? Smax : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            int h = (int)(r % Hq);
+            int b = (int)(r / Hq);
+            int hk = h / group;
+            int n = seqlens[b];
+            int lo = n - W < 0 ? 0 : n - W;
+            double ks = (double)k_descale[hk], vs = (double)v_descale[hk];
+            const uint16_t *qr = q + r * D;
+            double M = (double)sinks[h];
+            for (int t = lo; t < n; ++t) {
+                const uint8_t *kr = kc + (((int64_t)b * Smax + t) * Hkv + hk) * D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += bf16_to_f64(qr[d]) * (ks * e4m3_to_f64(kr[d]));
+                s[t - lo] = (double)scale * dot;
+                if (s[t - lo] > M) M = s[t - lo];
+            }
+            double *o = out + r * D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            double Z = (isinf((double)sinks[h]) && sinks[h] < 0) ? 0.0 : exp((double)sinks[h] - M);
+            for (int t = lo; t < n; ++t) {
+                double p = exp(s[t - lo] - M);
+                Z += p;
+                const uint8_t *vr = vc + (((int64_t)b * Smax + t) * Hkv + hk) * D;
+                for (int d = 0; d < D; ++d) o[d] += p * (vs * e4m3_to_f64(vr[d]));
+            }
+            if (Z > 0.0) {
+                for (int d = 0; d < D; ++d) o[d] /= Z;
+                if (lse) lse[r] = M + log(Z);
+            } else if (lse) {
+                lse[r] = -INFINITY;
+            }
+        }
+        free(s);
+    }
+    return 0;
+}
+
+/*
  * Split-KV step 1 (page 5, section 3): the partial softmax of one query row
  * over the keys [lo, hi] only, with no sink.  O_s is normalised within the
  * split and LSE_s is its natural-log normaliser.  Requires lo <= hi.
