@@ -46,7 +46,8 @@ extern "C" {
 enum attn_dtype {
     ATTN_DTYPE_BF16 = 1,
     ATTN_DTYPE_F32 = 2,
-    ATTN_DTYPE_I32 = 3
+    ATTN_DTYPE_I32 = 3,
+    ATTN_DTYPE_E4M3 = 4   /* FP8: 1 sign, 4 exponent (bias 7), 3 mantissa bits */
 };
 
 typedef struct attn_tensor {
@@ -195,6 +196,33 @@ int attn_sink_decode_paged(const attn_tensor *q, const attn_tensor *kpages,
                            const attn_tensor *vpages, const attn_tensor *block_table,
                            const attn_tensor *seqlens, const attn_tensor *sinks,
                            int32_t window, float scale, attn_tensor *out, void *stream);
+
+/*
+ * Single-token split-KV decode over an FP8 (e4m3) KV cache, dequantised per kv
+ * head (page "cf-1.com/news/6055759", "fix 2": the output scale is
+ * rcp(row_sum) * sink_rescale * v_descale; its FP8 max_offset belongs to an
+ * FP8 P, and P is not quantised here).
+ *
+ *   q          [B, Hq, D]        bf16, as for attn_sink_decode.
+ *   kcache,
+ *   vcache     [B, Smax, Hkv, D] ATTN_DTYPE_E4M3 bytes; every stride but the
+ *                                innermost a multiple of 16 elements.
+ *   k_descale,
+ *   v_descale  [Hkv] f32, DEVICE memory: key row = k_descale[hk] * e4m3(row),
+ *              value row likewise with v_descale.
+ *   seqlens, sinks, window, scale, out: as for attn_sink_decode.
+ *
+ * The same three launches as attn_sink_decode; the split kernel streams the
+ * e4m3 tiles (half the bytes of bf16), each consumer warp converts its keys
+ * to bf16 in shared memory (exact: every e4m3 value is a bf16 value) and the
+ * key descale is folded into the softmax scale.  D in {128, 256}; Hq/Hkv as
+ * for attn_sink_decode.
+ */
+int attn_sink_decode_fp8(const attn_tensor *q, const attn_tensor *kcache,
+                         const attn_tensor *vcache, const attn_tensor *k_descale,
+                         const attn_tensor *v_descale, const attn_tensor *seqlens,
+                         const attn_tensor *sinks, int32_t window, float scale,
+                         attn_tensor *out, void *stream);
 
 /*
  * attn_sink_decode without any allocation (the pages have no counterpart to

@@ -28,13 +28,15 @@ ATTN_ETIMEOUT = -5
 ATTN_DTYPE_BF16 = 1
 ATTN_DTYPE_F32 = 2
 ATTN_DTYPE_I32 = 3
+ATTN_DTYPE_E4M3 = 4
 
 _DTYPES = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float32: ATTN_DTYPE_F32,
-           torch.int32: ATTN_DTYPE_I32}
+           torch.int32: ATTN_DTYPE_I32, torch.float8_e4m3fn: ATTN_DTYPE_E4M3}
 
 # Every symbol include/attnsink.h declares.
 EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_varlen", "attn_sink_fwd_cudacore", "attn_sink_decode",
-           "attn_sink_decode_chunked", "attn_sink_decode_paged", "attn_sink_decode_noalloc",
+           "attn_sink_decode_chunked", "attn_sink_decode_paged", "attn_sink_decode_fp8",
+           "attn_sink_decode_noalloc",
            "attn_sink_get_status",
            "attn_sink_strerror", "attn_sink_last_error")
 
@@ -76,6 +78,8 @@ def load() -> ctypes.CDLL:
         lib.attn_sink_decode_chunked.restype = ctypes.c_int
         lib.attn_sink_decode_paged.argtypes = [P, P, P, P, P, P, i32, f32, P, V]
         lib.attn_sink_decode_paged.restype = ctypes.c_int
+        lib.attn_sink_decode_fp8.argtypes = [P, P, P, P, P, P, P, i32, f32, P, V]
+        lib.attn_sink_decode_fp8.restype = ctypes.c_int
         lib.attn_sink_decode_noalloc.argtypes = [P, P, P, P, P, i32, f32, P, V]
         lib.attn_sink_decode_noalloc.restype = ctypes.c_int
         lib.attn_sink_get_status.argtypes = [V]
@@ -198,6 +202,18 @@ def attn_sink_decode_paged(q, kpages, vpages, block_table, seqlens, sinks, windo
                                     _ref(ds[4]), _ref(ds[5]), int(window), float(scale),
                                     _ref(ds[6]), _stream(stream, q))
     _check(rc, "attn_sink_decode_paged")
+
+
+def attn_sink_decode_fp8(q, kcache, vcache, k_descale, v_descale, seqlens, sinks, window: int,
+                         scale: float, out, stream=None):
+    """C ``attn_sink_decode_fp8``: split-KV decode over an e4m3 cache
+    (``torch.float8_e4m3fn``) with per-kv-head descales ``[Hkv]`` (f32)."""
+    lib = load()
+    ds = [describe(x) for x in (q, kcache, vcache, k_descale, v_descale, seqlens, sinks, out)]
+    rc = lib.attn_sink_decode_fp8(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), _ref(ds[4]),
+                                  _ref(ds[5]), _ref(ds[6]), int(window), float(scale), _ref(ds[7]),
+                                  _stream(stream, q))
+    _check(rc, "attn_sink_decode_fp8")
 
 
 def attn_sink_decode_noalloc(q, kcache, vcache, seqlens, sinks, window: int, scale: float, out,

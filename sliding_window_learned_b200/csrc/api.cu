@@ -104,6 +104,7 @@ const char *dtype_name(int32_t d) {
     case ATTN_DTYPE_BF16: return "bf16";
     case ATTN_DTYPE_F32: return "f32";
     case ATTN_DTYPE_I32: return "i32";
+    case ATTN_DTYPE_E4M3: return "e4m3";
     default: return "unknown";
   }
 }
@@ -125,8 +126,10 @@ int check_tensor(const attn_tensor *t, const char *name, int32_t dtype, int ndim
     return fail(ATTN_EINVAL, "%s: innermost stride must be 1", name);
   for (int d = 0; d < ndim - 1; ++d) {
     if (t->stride[d] <= 0) return fail(ATTN_EINVAL, "%s: stride of dim %d must be positive", name, d);
-    if (tma && t->stride[d] % 8 != 0)
-      return fail(ATTN_EINVAL, "%s: stride of dim %d must be a multiple of 8 elements", name, d);
+    const int64_t per16 = dtype == ATTN_DTYPE_E4M3 ? 16 : 8;   // elements per 16 bytes
+    if (tma && t->stride[d] % per16 != 0)
+      return fail(ATTN_EINVAL, "%s: stride of dim %d must be a multiple of %lld elements (16 bytes)", name,
+                  d, (long long)per16);
   }
   return ATTN_OK;
 }
@@ -258,9 +261,9 @@ namespace {
 struct TmaKey {
   const void *base;
   int64_t d[4], s[3];
-  int box;
+  int box, elem;
   bool operator==(const TmaKey &o) const {
-    return base == o.base && box == o.box && memcmp(d, o.d, sizeof d) == 0 &&
+    return base == o.base && box == o.box && elem == o.elem && memcmp(d, o.d, sizeof d) == 0 &&
            memcmp(s, o.s, sizeof s) == 0;
   }
 };
@@ -277,7 +280,7 @@ std::mutex g_tma_mu;
 }  // namespace
 
 cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
-                          int64_t d0, const int64_t strides_el[3], int box_rows) {
+                          int64_t d0, const int64_t strides_el[3], int box_rows, int elem_bytes) {
   typedef CUresult (*encode_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -303,6 +306,7 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
   key.s[1] = strides_el[1];
   key.s[2] = strides_el[2];
   key.box = box_rows;
+  key.elem = elem_bytes;
   {
     std::lock_guard<std::mutex> lk(g_tma_mu);
     for (TmaEntry &e : g_tma_cache)
@@ -315,13 +319,16 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
                               static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
   // byte strides of dims 1..3 (innermost first): head, position, batch
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(strides_el[2]) * 2,
-                                 static_cast<cuuint64_t>(strides_el[1]) * 2,
-                                 static_cast<cuuint64_t>(strides_el[0]) * 2};
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(strides_el[2]) * eb,
+                                 static_cast<cuuint64_t>(strides_el[1]) * eb,
+                                 static_cast<cuuint64_t>(strides_el[0]) * eb};
+  // 128 bytes of the innermost dimension per box row (the swizzle span)
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   alignas(64) CUtensorMap map;
-  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+  const CUresult r = encode(&map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                            4, const_cast<void *>(base), dims,
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -489,6 +496,38 @@ int prep_decode_paged(const attn_tensor *q, const attn_tensor *kpages, const att
   return ATTN_OK;
 }
 
+// Validates the FP8-cache decode arguments: as prep_decode, with e4m3 caches
+// and the two [Hkv] f32 descale vectors.
+int prep_decode_fp8(const attn_tensor *q, const attn_tensor *kcache, const attn_tensor *vcache,
+                    const attn_tensor *k_descale, const attn_tensor *v_descale,
+                    const attn_tensor *seqlens, const attn_tensor *sinks, int32_t window, float scale,
+                    attn_tensor *out, DecodeArgs *out_args, bool *empty) {
+  int rc;
+  if ((rc = check_tensor(kcache, "kcache", ATTN_DTYPE_E4M3, 4, true))) return rc;
+  if ((rc = check_tensor(vcache, "vcache", ATTN_DTYPE_E4M3, 4, true))) return rc;
+  if ((rc = check_tensor(k_descale, "k_descale", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(v_descale, "v_descale", ATTN_DTYPE_F32, 1, false))) return rc;
+  const int64_t Hkv = kcache->shape[2], D = kcache->shape[3];
+  if (k_descale->shape[0] != Hkv || v_descale->shape[0] != Hkv)
+    return fail(ATTN_EINVAL, "k_descale and v_descale must have Hkv = %lld entries", (long long)Hkv);
+  if ((Hkv > 1 && (k_descale->stride[0] != 1 || v_descale->stride[0] != 1)))
+    return fail(ATTN_EINVAL, "descales must be contiguous");
+  if (D != 128 && D != 256) return fail(ATTN_EUNSUPPORTED, "FP8 cache: head dim %lld not supported (128, 256)", (long long)D);
+  // the remaining checks are those of the bf16 decode, on shape-only copies
+  attn_tensor kc = *kcache, vc = *vcache;
+  kc.dtype = vc.dtype = ATTN_DTYPE_BF16;
+  for (int d = 0; d < 3; ++d) {
+    if (kc.stride[d] % 16 != 0 || vc.stride[d] % 16 != 0)
+      return fail(ATTN_EINVAL, "FP8 cache strides must be multiples of 16 elements");
+  }
+  if ((rc = prep_decode(q, &kc, &vc, seqlens, sinks, window, scale, 0, out, out_args, empty))) return rc;
+  out_args->chunk = (out_args->chunk + 127) / 128 * 128;   // whole 128-key FP8 tiles
+  out_args->fp8 = true;
+  out_args->k_descale = static_cast<const float *>(k_descale->data);
+  out_args->v_descale = static_cast<const float *>(v_descale->data);
+  return ATTN_OK;
+}
+
 }  // namespace attnsink
 
 using namespace attnsink;
@@ -606,6 +645,31 @@ int attn_sink_decode_paged(const attn_tensor *q, const attn_tensor *kpages,
   e = launch_decode(a, ws, st);
   const cudaError_t ef = cudaFreeAsync(ws, st);
   if (e != cudaSuccess) return fail_cuda(e, "attn_sink_decode_paged launch");
+  if (ef != cudaSuccess) return fail_cuda(ef, "decode workspace release");
+  return ATTN_OK;
+}
+
+int attn_sink_decode_fp8(const attn_tensor *q, const attn_tensor *kcache, const attn_tensor *vcache,
+                         const attn_tensor *k_descale, const attn_tensor *v_descale,
+                         const attn_tensor *seqlens, const attn_tensor *sinks, int32_t window,
+                         float scale, attn_tensor *out, void *stream) {
+  t_last_error[0] = '\0';
+  DecodeArgs a;
+  bool empty;
+  int rc = prep_decode_fp8(q, kcache, vcache, k_descale, v_descale, seqlens, sinks, window, scale, out, &a,
+                           &empty);
+  if (rc || empty) return rc;
+  if ((rc = status_ptr(&a.status))) return rc;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  const size_t bytes = decode_workspace_bytes(a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void *ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, st);
+  if (e != cudaSuccess) return fail_cuda(e, "decode workspace allocation");
+  e = launch_decode(a, ws, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e != cudaSuccess) return fail_cuda(e, "attn_sink_decode_fp8 launch");
   if (ef != cudaSuccess) return fail_cuda(ef, "decode workspace release");
   return ATTN_OK;
 }

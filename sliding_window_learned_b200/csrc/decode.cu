@@ -38,10 +38,8 @@
 namespace attnsink {
 namespace {
 
-constexpr int kTK = 64;               // keys per tile
-constexpr int kConsumerWarps = 4;     // each owns 16 keys of every tile
-constexpr int kProducerWarp = 4;
-constexpr int kThreads = 5 * 32;
+constexpr int kTK = 64;               // keys per tile (bf16 cache)
+constexpr int kConsumerWarps = 4;     // each owns 16 keys of every tile (bf16 cache)
 constexpr uint32_t kBarMerge = 1;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -138,6 +136,9 @@ struct SplitParams {
   const int *block_table;
   int64_t bt_s0;
   int page, page_shift, max_pages, align;
+  // FP8 e4m3 cache: per-kv-head dequantisation scales (key row = k_descale *
+  // e4m3 row; v_descale scales the partial output)
+  const float *k_descale, *v_descale;
 };
 
 struct StageInfo {
@@ -146,17 +147,58 @@ struct StageInfo {
   int pad;
 };
 
-template <int D, int NT>
+// kF8: the cache holds FP8 e4m3 bytes.  Its tiles arrive in 128-byte
+// (128-element) swizzled chunks; each consumer warp converts its 16 keys of K
+// and V to f16 (one cvt per pair, exact) into a tile of the 16-bit layout
+// (kConvBytes), and the MMA code below runs on that tile in f16: q is
+// converted to f16 after a power-of-two scale that puts its largest magnitude
+// in [2^13, 2^14) (undone in the softmax scale), and P is f16.
+// An FP8 cache delivers a key in half the bytes, so at D = 128 its tiles are
+// 128 keys for 8 consumer warps (two per SM sub-partition), which keeps the
+// consumers ahead of HBM; the merge buffer then lives in the conversion tile
+// (free at an item's end).
+template <int D, int NT, bool kF8>
 struct DCfg {
-  static constexpr int kChunks = D / 64;
-  static constexpr int kTileBytes = kTK * D * 2;          // one K (or V) tile
+  static constexpr int kCW = (kF8 && D == 128) ? 8 : kConsumerWarps;   // consumer warps
+  static constexpr int kTK = 16 * kCW;                    // keys per tile
+  static constexpr int kThreads = (kCW + 1) * 32;         // + the producer warp
+  static constexpr bool kMergeInConv = kF8;
+  static constexpr int kChunks = D / 64;                  // 64-element chunks of a bf16 row
+  static constexpr int kChunks8 = D / 128;                // 128-element chunks of an FP8 row
+  static constexpr int kTileBytes = kTK * D * (kF8 ? 1 : 2);   // one K (or V) tile as stored
+  static constexpr int kBf16TileBytes = kTK * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
-  static constexpr int kStages = (196608 / kStageBytes) > 12 ? 12 : (196608 / kStageBytes);
-  static constexpr int kMergeBytes = kConsumerWarps * NT * 8 * D * 4;
-  static constexpr int kInfoOffset = kStages * kStageBytes + kMergeBytes;
-  static constexpr int kSmemBytes = kInfoOffset + 1024 + 1024;
+  static constexpr int kConvBytes = kF8 ? 2 * kBf16TileBytes : 0;
+  static constexpr int kMergeBytes = kCW * NT * 8 * D * 4;
+  static constexpr int kRingBudget = 196608 - kConvBytes - (kMergeInConv ? 0 : kMergeBytes);
+  static constexpr int kStages = (kRingBudget / kStageBytes) > 12 ? 12 : (kRingBudget / kStageBytes);
+  static constexpr int kConvOffset = kStages * kStageBytes;
+  static constexpr int kMergeOffset = kMergeInConv ? kConvOffset : kConvOffset + kConvBytes;
+  static constexpr int kInfoOffset = kConvOffset + kConvBytes + (kMergeInConv ? 0 : kMergeBytes);
+  static_assert(!kMergeInConv || kMergeBytes <= kConvBytes, "merge buffer fits the conversion tile");
+  // stage descriptors, full/empty barriers, per-warp (max, sum) for the merge,
+  // the abort flag; plus 1 KB of slack for aligning the base to 1 KB
+  static constexpr int kInfoBytes =
+      (kStages * 32 + kStages * 16 + 2 * kCW * NT * 8 * 4 + 16 + 127) / 128 * 128;
+  static constexpr int kSmemBytes = kInfoOffset + kInfoBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(!kF8 || D % 128 == 0, "FP8 rows are whole 128-byte chunks");
 };
+
+// Two e4m3 values (low byte first) to an f16 pair: one cvt, exact (every
+// e4m3 value, subnormals included, is a normal f16; NaN stays NaN).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+  uint32_t h;
+  asm("{.reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t;}" : "=r"(h) : "r"(two_bytes));
+  return h;
+}
+
+// bf16 pair -> f16 pair times a power of two (exact unless the product falls
+// below the f16 normal range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x, float s) {
+  const float lo = __uint_as_float(x << 16) * s, hi = __uint_as_float(x & 0xFFFF0000u) * s;
+  return pack_f16x2(lo, hi);
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const WaitCtx &ctx,
                                           int where) {
@@ -164,21 +206,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, r);
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int NT, bool kF8>
+__global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const SplitParams p) {
-  using C = DCfg<D, NT>;
+  using C = DCfg<D, NT, kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  float *merge = reinterpret_cast<float *>(smem + C::kStages * C::kStageBytes);
+  float *merge = reinterpret_cast<float *>(smem + C::kMergeOffset);
   StageInfo *info = reinterpret_cast<StageInfo *>(smem + C::kInfoOffset);
   uint64_t *full = reinterpret_cast<uint64_t *>(info + C::kStages);
   uint64_t *empty = full + C::kStages;
   float *merge_m = reinterpret_cast<float *>(empty + C::kStages);   // [4][NT*8]
-  float *merge_l = merge_m + kConsumerWarps * NT * 8;               // [4][NT*8]
-  int *abort_flag = reinterpret_cast<int *>(merge_l + kConsumerWarps * NT * 8);
+  float *merge_l = merge_m + C::kCW * NT * 8;               // [4][NT*8]
+  int *abort_flag = reinterpret_cast<int *>(merge_l + C::kCW * NT * 8);
   const WaitCtx ctx{abort_flag, p.status};
 
   const int warp = threadIdx.x >> 5;
@@ -186,14 +228,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], C::kCW);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kProducerWarp) {
+  if (warp == C::kCW) {
     // -------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
@@ -224,8 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int vis0 = max(0, n - p.W);
         const int ks = vis0 / p.align * p.align + split * p.chunk;
         const int ke = min(n, ks + p.chunk);
-        const int nt = (ke - ks + kTK - 1) / kTK;
-        const int nbox = p.page == 0 ? 1 : kTK / min(kTK, p.page);   // boxes per tile (paged)
+        const int nt = (ke - ks + C::kTK - 1) / C::kTK;
+        const int nbox = p.page == 0 ? 1 : C::kTK / min(C::kTK, p.page);   // boxes per tile (paged)
         for (int t = 0; ok && t < nt; ++t) {
           // Paged cache: read the tile's page numbers before waiting for a free
           // stage, so that the table reads overlap the wait.
@@ -234,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
               if (r >= nbox) break;
-              const int lp = (ks + t * kTK + r * (kTK / nbox)) >> p.page_shift;
+              const int lp = (ks + t * C::kTK + r * (C::kTK / nbox)) >> p.page_shift;
               blk[r] = lp < p.max_pages ? p.block_table[static_cast<int64_t>(b) * p.bt_s0 + lp] : -1;
             }
           }
@@ -244,16 +286,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           si.b = b;
           si.hk = hk;
           si.split = split;
-          si.key0 = ks + t * kTK;
-          si.nvalid = min(kTK, ke - si.key0);
+          si.key0 = ks + t * C::kTK;
+          si.nvalid = min(C::kTK, ke - si.key0);
           si.nskip = max(0, vis0 - si.key0);
           si.flags = (t == 0 ? 1 : 0) | (t == nt - 1 ? 2 : 0);
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
           uint8_t *dst = smem + s * C::kStageBytes;
-          if (p.page == 0) {
+          if (kF8) {
+            for (int c = 0; c < C::kChunks8; ++c) {
+              tma_load_4d(dst + c * C::kTK * 128, &tmK, &full[s], c * 128, hk, si.key0, b);
+              tma_load_4d(dst + C::kTileBytes + c * C::kTK * 128, &tmV, &full[s], c * 128, hk, si.key0, b);
+            }
+          } else if (p.page == 0) {
             for (int c = 0; c < C::kChunks; ++c) {
-              tma_load_4d(dst + c * kTK * 128, &tmK, &full[s], c * 64, hk, si.key0, b);
-              tma_load_4d(dst + C::kTileBytes + c * kTK * 128, &tmV, &full[s], c * 64, hk, si.key0, b);
+              tma_load_4d(dst + c * C::kTK * 128, &tmK, &full[s], c * 64, hk, si.key0, b);
+              tma_load_4d(dst + C::kTileBytes + c * C::kTK * 128, &tmV, &full[s], c * 64, hk, si.key0, b);
             }
           } else {
             // key0 is a multiple of 64 here, so each box of min(64, page) rows
@@ -261,15 +308,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // number past the table, for rows beyond the sequence end) loads
             // zero rows: the box is out of range and filled, and it still
             // delivers its bytes.
-            const int rows = kTK / nbox;
+            const int rows = C::kTK / nbox;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
               if (r >= nbox) break;
               const int r0 = r * rows;
               const int slot = (si.key0 + r0) & (p.page - 1);
               for (int c = 0; c < C::kChunks; ++c) {
-                tma_load_4d(dst + c * kTK * 128 + r0 * 128, &tmK, &full[s], c * 64, hk, slot, blk[r]);
-                tma_load_4d(dst + C::kTileBytes + c * kTK * 128 + r0 * 128, &tmV, &full[s], c * 64, hk,
+                tma_load_4d(dst + c * C::kTK * 128 + r0 * 128, &tmK, &full[s], c * 64, hk, slot, blk[r]);
+                tma_load_4d(dst + C::kTileBytes + c * C::kTK * 128 + r0 * 128, &tmV, &full[s], c * 64, hk,
                             slot, blk[r]);
               }
             }
@@ -291,7 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------- consumers
   const int g8 = lane >> 2;       // mma "group" (row within an 8-row block)
   const int tig = lane & 3;       // thread in group
-  const float sl2 = p.scale_log2;
+  float sl2 = p.scale_log2;       // (FP8: times the item's key descale)
+  float vdesc = 1.f;              // (FP8: the item's value descale)
   uint32_t qf[D / 16][NT][2];     // B fragments of q^T, per k-step and head tile
   float o[D / 16][NT][4];         // O^T accumulators: [d tile][head tile][frag]
   float m_run[NT][2], l_run[NT][2];
@@ -302,8 +350,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     ++slot;
     const StageInfo si = info[s];
     if (si.flags & 4) break;
-    const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
-    const uint32_t vbase = kbase + C::kTileBytes;
+    const int key_w = warp * 16;  // this warp's 16 keys within the tile
+    uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
+    uint32_t vbase = kbase + C::kTileBytes;
+    if constexpr (kF8) {
+      // This warp's 16 K and V rows, e4m3 -> f16, into the conversion tile
+      // (the layout of a 16-bit stage); rows outside [nskip, nvalid) become
+      // zeros.  Then the FP8 stage goes back to the producer at once.
+      const uint8_t *src = smem + s * C::kStageBytes;
+      uint8_t *conv = smem + C::kConvOffset;
+      const int row = key_w + (lane >> 1);
+      const bool valid = row >= si.nskip && row < si.nvalid;
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+#pragma unroll
+        for (int c8 = 0; c8 < C::kChunks8; ++c8) {
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            const int u = (lane & 1) * 4 + uu;     // 16-byte unit (16 elements) of the 128-byte row
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (valid)
+              x = *reinterpret_cast<const uint4 *>(src + kv * C::kTileBytes + c8 * C::kTK * 128 + row * 128 +
+                                                   ((u ^ (row & 7)) << 4));
+            uint4 lo, hi;                          // elements 0..7 and 8..15 as f16
+            lo.x = e4m3x2_to_f16x2(x.x & 0xFFFFu);
+            lo.y = e4m3x2_to_f16x2(x.x >> 16);
+            lo.z = e4m3x2_to_f16x2(x.y & 0xFFFFu);
+            lo.w = e4m3x2_to_f16x2(x.y >> 16);
+            hi.x = e4m3x2_to_f16x2(x.z & 0xFFFFu);
+            hi.y = e4m3x2_to_f16x2(x.z >> 16);
+            hi.z = e4m3x2_to_f16x2(x.w & 0xFFFFu);
+            hi.w = e4m3x2_to_f16x2(x.w >> 16);
+            const int col = c8 * 128 + u * 16;     // first element of this unit
+            const int cb = col >> 6, ub = (col & 63) >> 3;
+            uint8_t *drow = conv + kv * C::kBf16TileBytes + cb * C::kTK * 128 + row * 128;
+            *reinterpret_cast<uint4 *>(drow + ((ub ^ (row & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4 *>(drow + (((ub + 1) ^ (row & 7)) << 4)) = hi;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      kbase = smem_u32(conv);
+      vbase = kbase + C::kBf16TileBytes;
+    }
     if (si.flags & 1) {
       // first tile of a work item: load this kv head's grouped queries
 #pragma unroll
@@ -331,16 +421,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run[nt][0] = m_run[nt][1] = -INFINITY;
         l_run[nt][0] = l_run[nt][1] = 0.f;
       }
+      if constexpr (kF8) {
+        // q to f16 with a power-of-two scale 2^e that puts max|q| in
+        // [2^13, 2^14): exact for every q element above max|q| * 2^-27;
+        // 2^-e then joins the softmax scale with the key descale
+        float mx = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int f = 0; f < 2; ++f) {
+              const uint32_t x = qf[kk][nt][f];
+              mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(x << 16)), fabsf(__uint_as_float(x & 0xFFFF0000u))));
+            }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        int e = 0;
+        if (mx > 0.f && mx < INFINITY) e = 13 - ilogbf(mx);
+        const float qs = ldexpf(1.f, e);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int f = 0; f < 2; ++f) qf[kk][nt][f] = bf16x2_to_f16x2_scaled(qf[kk][nt][f], qs);
+        sl2 = p.scale_log2 * p.k_descale[si.hk] * ldexpf(1.f, -e);
+        vdesc = p.v_descale[si.hk];
+      }
     }
-    const int key_w = warp * 16;  // this warp's 16 keys within the tile
     // Keys past the end of the split, and (paged cache) keys before the
     // window, are masked; their cache rows may hold anything (NaN included),
     // so their V rows are zeroed in shared memory before P.V reads them.
-    if (si.nvalid < key_w + 16 || si.nskip > key_w) {
+    if (!kF8 && (si.nvalid < key_w + 16 || si.nskip > key_w)) {
       const int kidx = key_w + (lane & 15);
       if (kidx >= si.nvalid || kidx < si.nskip) {
         for (int c = 0; c < C::kChunks; ++c) {
-          uint8_t *row = smem + s * C::kStageBytes + C::kTileBytes + c * kTK * 128 + kidx * 128;
+          uint8_t *row = smem + s * C::kStageBytes + C::kTileBytes + c * C::kTK * 128 + kidx * 128;
           const int half = lane >> 4;
 #pragma unroll
           for (int u = 0; u < 4; ++u)
@@ -360,11 +477,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const int unit = 2 * (kk & 3) + (lane >> 4);
-        const uint32_t addr = kbase + (kk >> 2) * (kTK * 128) + krow * 128 + ((unit ^ (krow & 7)) << 4);
+        const uint32_t addr = kbase + (kk >> 2) * (C::kTK * 128) + krow * 128 + ((unit ^ (krow & 7)) << 4);
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4(addr, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if constexpr (kF8)
+            mma_f16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+          else
+            mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+        }
       }
     }
     // ---- online softmax per head (no sink here) ----
@@ -405,8 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // P^T fragments (key rows, head columns) -> transposed into the
       // B-operand layout of O^T += V^T P^T.
-      pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-      pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+      pb[nt][0] = movmatrix_trans(kF8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1));
+      pb[nt][1] = movmatrix_trans(kF8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3));
     }
     // ---- O^T[D x 8*NT] += V_w^T P^T ----
     {
@@ -414,18 +536,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int dm = 0; dm < D / 16; ++dm) {
         const int unit = 2 * (dm & 3) + ((lane >> 3) & 1);
-        const uint32_t addr = vbase + (dm >> 2) * (kTK * 128) + vrow * 128 + ((unit ^ (vrow & 7)) << 4);
+        const uint32_t addr = vbase + (dm >> 2) * (C::kTK * 128) + vrow * 128 + ((unit ^ (vrow & 7)) << 4);
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(addr, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if constexpr (kF8)
+            mma_f16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          else
+            mma_bf16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        }
       }
     }
     // release the stage (generic-proxy writes above are ordered before the
-    // next TMA write into it)
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    // next TMA write into it); an FP8 stage was released after conversion
+    if constexpr (!kF8) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    } else {
+      __syncwarp();   // the conversion tile is rewritten only after every lane's MMAs
+    }
 
     if (si.flags & 2) {
       // ---- merge the four warps' partial states and write (O_s, LSE_s) ----
@@ -438,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
           l_run[nt][e] = l;
         }
-      named_barrier_sync(kBarMerge, kConsumerWarps * 32);  // previous merge fully read
+      named_barrier_sync(kBarMerge, C::kCW * 32);  // previous merge fully read
       if (g8 == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -459,17 +590,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mw[hh * D + dm * 16 + g8 + 8] = o[dm][nt][2];
           mw[(hh + 1) * D + dm * 16 + g8 + 8] = o[dm][nt][3];
         }
-      named_barrier_sync(kBarMerge, kConsumerWarps * 32);
-      const int tid = threadIdx.x;  // 0..127
+      named_barrier_sync(kBarMerge, C::kCW * 32);
+      const int tid = threadIdx.x;  // 0 .. consumer threads - 1
       const int gsplit = p.base[si.b] + si.split;
-      for (int e = tid; e < p.G * D; e += kConsumerWarps * 32) {
+      for (int e = tid; e < p.G * D; e += C::kCW * 32) {
         const int hh = e / D, d = e - hh * D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w * NT * 8 + hh]);
+        for (int w = 0; w < C::kCW; ++w) M = fmaxf(M, merge_m[w * NT * 8 + hh]);
         float num = 0.f, den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < C::kCW; ++w) {
           const float mw_ = merge_m[w * NT * 8 + hh];
           const float f = (mw_ == -INFINITY) ? 0.f : ex2_approx(mw_ - M);
           num += f * merge[w * (NT * 8 * D) + hh * D + d];
@@ -477,9 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int hq = si.hk * p.G + hh;
         const size_t row = static_cast<size_t>(gsplit) * p.Hq + hq;
-        p.o_part[row * D + d] = num / den;
+        p.o_part[row * D + d] = num / den * vdesc;
         if (d == 0) p.lse_part[row] = (M + log2f(den)) * kLn2;
       }
+      // the merge buffer is the conversion tile: every reader is done before
+      // any warp converts the next tile into it
+      if constexpr (C::kMergeInConv) named_barrier_sync(kBarMerge, C::kCW * 32);
     }
   }
 }
@@ -555,16 +689,19 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const int *nsplit, 
   for (int t = 0; t < DPL; ++t) orow[lane + 32 * t] = __float2bfloat16_rn(acc[t] * inv);
 }
 
-template <int D, int NT>
+template <int D, int NT, bool kF8>
 cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cudaStream_t stream) {
-  using C = DCfg<D, NT>;
+  using C = DCfg<D, NT, kF8>;
   alignas(64) CUtensorMap mk, mv;
   cudaError_t e;
-  if (a.page == 0) {
-    if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, kTK)) != cudaSuccess) return e;
-    if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, kTK)) != cudaSuccess) return e;
+  if (kF8) {
+    if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, C::kTK, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, C::kTK, 1)) != cudaSuccess) return e;
+  } else if (a.page == 0) {
+    if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, C::kTK)) != cudaSuccess) return e;
+    if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, C::kTK)) != cudaSuccess) return e;
   } else {
-    const int rows = a.page < kTK ? a.page : kTK;
+    const int rows = a.page < C::kTK ? a.page : C::kTK;
     if ((e = make_tma_bshd(&mk, a.kc, a.npages, a.page, a.Hkv, D, a.kc_s, rows)) != cudaSuccess) return e;
     if ((e = make_tma_bshd(&mv, a.vc, a.npages, a.page, a.Hkv, D, a.vc_s, rows)) != cudaSuccess) return e;
   }
@@ -594,18 +731,20 @@ cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cu
   p.page_shift = 0;
   while (a.page > 0 && (1 << p.page_shift) < a.page) ++p.page_shift;
   p.max_pages = a.max_pages;
-  p.align = a.page > 0 ? kTK : 1;
+  p.align = a.page > 0 ? C::kTK : 1;
+  p.k_descale = a.k_descale;
+  p.v_descale = a.v_descale;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const long long items = static_cast<long long>(w.max_splits) * a.Hkv;
   const int grid = static_cast<int>(items < sms ? items : sms);
   if (grid <= 0) return cudaSuccess;
-  auto kern = decode_split_kernel<D, NT>;
+  auto kern = decode_split_kernel<D, NT, kF8>;
   if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes)) !=
       cudaSuccess)
     return e;
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(mk, mv, p);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, p);
   return cudaGetLastError();
 }
 
@@ -642,9 +781,20 @@ cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t str
   if (e != cudaSuccess) return e;
   const int G = a.Hq / a.Hkv;
   switch (a.D) {
-    case 64: e = G <= 8 ? launch_split<64, 1>(a, w, ws, stream) : launch_split<64, 2>(a, w, ws, stream); break;
-    case 128: e = G <= 8 ? launch_split<128, 1>(a, w, ws, stream) : launch_split<128, 2>(a, w, ws, stream); break;
-    case 256: e = G <= 8 ? launch_split<256, 1>(a, w, ws, stream) : cudaErrorInvalidValue; break;
+    case 64:
+      e = a.fp8 ? cudaErrorInvalidValue
+                : (G <= 8 ? launch_split<64, 1, false>(a, w, ws, stream) : launch_split<64, 2, false>(a, w, ws, stream));
+      break;
+    case 128:
+      if (a.fp8)
+        e = G <= 8 ? launch_split<128, 1, true>(a, w, ws, stream) : launch_split<128, 2, true>(a, w, ws, stream);
+      else
+        e = G <= 8 ? launch_split<128, 1, false>(a, w, ws, stream) : launch_split<128, 2, false>(a, w, ws, stream);
+      break;
+    case 256:
+      if (G > 8) e = cudaErrorInvalidValue;
+      else e = a.fp8 ? launch_split<256, 1, true>(a, w, ws, stream) : launch_split<256, 1, false>(a, w, ws, stream);
+      break;
     default: e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

@@ -47,6 +47,9 @@ struct DecodeArgs {
   int64_t bt_s0 = 0;
   int page = 0;                            // 0: contiguous cache; else a power of two >= 16
   int npages = 0, max_pages = 0;
+  // FP8 e4m3 cache (contiguous only): per-kv-head dequantisation scales
+  bool fp8 = false;
+  const float *k_descale = nullptr, *v_descale = nullptr;
 };
 
 // Bytes of stream-ordered workspace one decode call needs (256-byte aligned
@@ -63,7 +66,9 @@ cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t str
 // contiguous) with 128-byte swizzle and a box of {64, 1, box_rows, 1}, i.e.
 // box_rows consecutive positions of one head and 64 of its channels.
 // Returns cudaErrorInvalidValue if the driver rejects the description.
+// elem_bytes = 1 describes a byte tensor (FP8) instead, with a box of
+// {128, 1, box_rows, 1}: 128 one-byte elements per 128-byte swizzled row.
 cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
-                          int64_t d0, const int64_t strides_el[3], int box_rows);
+                          int64_t d0, const int64_t strides_el[3], int box_rows, int elem_bytes = 2);
 
 }  // namespace attnsink
