@@ -10,7 +10,8 @@ L2 (the prefill inputs are smaller than L2; the decode cache is ~17 GB).
 ranks, from CUDA events around each prefill launch; the decode figure (HBM
 GB/s of algorithmic bytes) is reported beside it, and after the timed steps
 the same decode over a paged copy of its cache (256-position pages at random
-pool positions, attn_sink_decode_paged) is timed as `decode_paged`, and the
+pool positions, attn_sink_decode_paged) is timed as `decode_paged`, the decode
+over the cache quantised to e4m3 (attn_sink_decode_fp8) as `decode_fp8`, and the
 forward over a seeded mix of 24 packed sequences (attn_sink_fwd_varlen) as
 `fwd_varlen`.
 `--impl reference` times
@@ -265,6 +266,36 @@ def run_ours(args, rank, world, local_rank):
     t_paged = e0.elapsed_time(e1) / 1e3
     del kpool, vpool, table
 
+    # ---- the same decode over its cache quantised to FP8 e4m3 per kv head ----
+    kdesc = torch.empty(dcfg.Hkv, device=dev)
+    vdesc = torch.empty(dcfg.Hkv, device=dev)
+    k8 = torch.empty(y["kcache"].shape, dtype=torch.float8_e4m3fn, device=dev)
+    v8 = torch.empty_like(k8)
+    for hk in range(dcfg.Hkv):
+        for src, dst, dsc in ((y["kcache"], k8, kdesc), (y["vcache"], v8, vdesc)):
+            xs = src[:, :, hk].float()
+            dsc[hk] = torch.nan_to_num(xs, nan=0.0).abs().amax() / 448.0
+            dst[:, :, hk] = (xs / dsc[hk]).to(torch.float8_e4m3fn)
+            del xs
+
+    def dec_fp8():
+        swl.attn_sink_decode_fp8(y["q"], k8, v8, kdesc, vdesc, y["seqlens"], y["sinks"], dcfg.W,
+                                 dcfg.scale, dout, stream)
+
+    for _ in range(3):
+        dec_fp8()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Kp):
+        dec_fp8()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if swl.attn_sink_get_status() != 0:
+        raise RuntimeError("device status error in the FP8 decode")
+    t_fp8 = e0.elapsed_time(e1) / 1e3
+    dbytes8 = (dbytes - 2 * dcfg.B * dcfg.Hq * dcfg.D * 2) // 2 + 2 * dcfg.B * dcfg.Hq * dcfg.D * 2
+    del k8, v8
+
     # ---- the forward over packed variable-length sequences: a seeded mix of
     # 24 sequences of U[1, 4096] tokens at the prefill workload's heads ----
     vl_rng = np.random.default_rng(1000 + rank)
@@ -301,10 +332,11 @@ def run_ours(args, rank, world, local_rank):
     del vq, vk, vv, vout, vlse
 
     # ---- max over ranks ----
-    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen], dtype=torch.float64, device=dev)
+    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8], dtype=torch.float64,
+                         device=dev)
     if world > 1:
         dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen = times.tolist()
+    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8 = times.tolist()
 
     if rank != 0:
         return
@@ -353,6 +385,11 @@ def run_ours(args, rank, world, local_rank):
                          "frac": round(dbytes / (t_paged / Kp) / 1e9 / hbm_peak, 4),
                          "what": "attn_sink_decode_paged on the decode workload, cache in 256-position "
                                  "pages at random pool positions"},
+        "decode_fp8": {"value": round(world * Kp * dbytes8 / t_fp8 / 1e9, 2), "unit": "GB/s",
+                       "ms_per_call": round(t_fp8 / Kp * 1e3, 4),
+                       "frac": round(dbytes8 / (t_fp8 / Kp) / 1e9 / hbm_peak, 4),
+                       "what": "attn_sink_decode_fp8 on the decode workload, cache quantised to e4m3 per "
+                               "kv head (bytes counted at one per element)"},
         "fwd_varlen": {"value": round(world * Kv * vl_flops / t_varlen / 1e12, 3), "unit": "TFLOP/s",
                        "ms_per_call": round(t_varlen / Kv * 1e3, 5),
                        "frac": round(vl_flops / (t_varlen / Kv) / 1e12 / bf16_peak, 4),
