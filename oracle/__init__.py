@@ -134,6 +134,36 @@ def fwd_varlen(q, k, v, cu_seqlens, sinks, window: int, scale: float):
     return out, lse
 
 
+def max_logit(q, k, window: int, scale: float):
+    """The largest pre-softmax logit of every (batch, query head): the maximum
+    over rows i and visible keys j in [max(0, i-W+1), i] of scale * <q_i, k_j>
+    (kv head h // (Hq/Hkv)), the sink excluded (the flash-attention contributor
+    guide's task for issue #2986: per-head maxima of shape (batch, nheads)).
+    q [B,L,Hq,D], k [B,L,Hkv,D] as uint16 bf16 bits.  Returns [B, Hq] float64
+    (-inf where L = 0).  Plain fp64, one key offset of the window at a time."""
+    q, k = _u16(q), _u16(k)
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    qd = _bits_to_f64(q)
+    kd = _bits_to_f64(k)
+    group = Hq // Hkv
+    out = np.full((B, Hq), -np.inf)
+    for h in range(Hq):
+        qh = qd[:, :, h, :]                       # [B, L, D]
+        kh = kd[:, :, h // group, :]
+        for off in range(min(window, L)):         # key j = i - off
+            if off >= L:
+                break
+            s = float(scale) * np.einsum("bld,bld->bl", qh[:, off:], kh[:, :L - off])
+            out[:, h] = np.maximum(out[:, h], s.max(axis=1))
+    return out
+
+
+def _bits_to_f64(a: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) to float64, exactly."""
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def fwd_rows(q, k, v, sinks, window: int, scale: float, rows):
     """The forward for selected rows only.  rows: int array [n, 3] of
     (b, i, h).  Returns (out [n, D] float64, lse [n] float64)."""
