@@ -88,6 +88,24 @@ int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
                   attn_tensor *out, attn_tensor *lse, void *stream);
 
 /*
+ * attn_sink_fwd that also returns the largest pre-softmax logit of every
+ * (batch, query head): max over rows i and visible keys j of
+ * scale * <q_i, k_j>, the sink excluded (page "Dao-AILab/flash-attention"
+ * contributor guide, task for issue #2986: expose the maximum pre-softmax
+ * logit, per-head maxima of shape (batch, nheads), from the running row
+ * maxima the kernel already keeps).
+ *
+ *   max_logit  [B, Hq] f32 (innermost stride 1), written completely: -inf
+ *              where a (batch, head) has no position (L = 0).
+ * Everything else as attn_sink_fwd.  The maxima come from the same fp32
+ * scores the softmax uses.
+ */
+int attn_sink_fwd_max_logit(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                            const attn_tensor *sinks, int32_t window, float scale,
+                            attn_tensor *out, attn_tensor *lse, attn_tensor *max_logit,
+                            void *stream);
+
+/*
  * Prefill forward over packed variable-length sequences (the varlen path of
  * page "Dao-AILab/flash-attention" contributor guide, call walk-through step
  * 2: cu_seqlens turned into per-sequence query tiles), with the learned sink

@@ -563,6 +563,32 @@ int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
   return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd launch");
 }
 
+int attn_sink_fwd_max_logit(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                            const attn_tensor *sinks, int32_t window, float scale, attn_tensor *out,
+                            attn_tensor *lse, attn_tensor *max_logit, void *stream) {
+  t_last_error[0] = '\0';
+  FwdArgs a;
+  int rc = prep_fwd(q, k, v, sinks, window, scale, out, lse, true, &a);
+  if (rc) return rc;
+  if (a.D != 64 && a.D != 128 && a.D != 256)
+    return fail(ATTN_EUNSUPPORTED, "head dim %d not supported (64, 128, 256)", a.D);
+  if ((rc = check_tensor(max_logit, "max_logit", ATTN_DTYPE_F32, 2, false))) return rc;
+  if (max_logit->shape[0] != a.B || max_logit->shape[1] != a.Hq)
+    return fail(ATTN_EINVAL, "max_logit must be [B, Hq]");
+  if (a.B == 0 || a.Hq == 0) return ATTN_OK;
+  a.max_logit = static_cast<float *>(max_logit->data);
+  a.ml_sb = max_logit->stride[0];
+  if (a.L == 0) {
+    // no position anywhere: every maximum is -inf and there is nothing else
+    const cudaError_t e = launch_max_logit_init(a.max_logit, a.ml_sb, a.B, a.Hq,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd_max_logit launch");
+  }
+  if ((rc = status_ptr(&a.status))) return rc;
+  const cudaError_t e = launch_fwd_tc(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_fwd_max_logit launch");
+}
+
 int attn_sink_fwd_varlen(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
                          const attn_tensor *cu_seqlens, int32_t max_seqlen,
                          const attn_tensor *sinks, int32_t window, float scale, attn_tensor *out,

@@ -124,6 +124,8 @@ struct Params {
   int T;
   __nv_bfloat16 *out;
   int64_t o_sr, o_sh;
+  float *max_logit;                        // [B, Hq] (stride ml_sb), kMaxLogit only
+  int64_t ml_sb;
 };
 
 // Warp-uniform bounded wait: every lane learns the same outcome, so the
@@ -296,6 +298,7 @@ template <int D, int BN>
 __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col, uint32_t o_col,
                                              int j, int g, float sl2, int lo, int hi, uint32_t cls_mask,
                                              uint32_t cls_none, float &m_run, float &l_run,
+                                             float &row_max,
                                              uint64_t *pv_done,
                                              const WaitCtx &ctx) {
   constexpr int NC = BN / 32;
@@ -311,6 +314,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col,
   if (j == 0) {
     // first tile: nothing accumulated yet, so take the maximum first
     const float mt2 = tile_max<BN>(sv, cls_none) * sl2;
+    row_max = fmaxf(row_max, mt2);
     if (mt2 > m_run + kRescaleThreshold) m_run = mt2;
     l_run = exp_tile<BN, false>(sv, lane_base + s_col, sl2, (m_run == -INFINITY) ? 0.f : m_run,
                                 cls_none, tm);
@@ -323,6 +327,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col,
   // maximum is taken now (and usually turns out not to have moved either).
   if (!kFusedMax) tm = (sum <= 256.f) ? -INFINITY : tile_max<BN>(sv, cls_none);
   const float mt2 = tm * sl2;
+  row_max = fmaxf(row_max, mt2);
   const bool grow = mt2 > m_run + kRescaleThreshold;
   if (!__any_sync(0xffffffffu, grow)) {
     l_run += sum;
@@ -356,7 +361,24 @@ __device__ __forceinline__ bool softmax_tile(uint32_t lane_base, uint32_t s_col,
 
 // kPacked: packed variable-length sequences (Params::cu_seqlens); a separate
 // instantiation, so that the batched kernel carries none of its code.
-template <int D, int BN, int NH, bool kPacked>
+__global__ void max_logit_init_kernel(float *ml, int64_t sb, int B, int Hq) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < B * Hq) ml[static_cast<int64_t>(t / Hq) * sb + t % Hq] = -INFINITY;
+}
+
+// Float maximum by integer atomics: non-negative floats order as signed ints,
+// negative ones in reverse as unsigned ints (so -inf, the start value, loses
+// to every other value).
+__device__ __forceinline__ void atomic_max_float(float *addr, float v) {
+  if (v >= 0.f)
+    atomicMax(reinterpret_cast<int *>(addr), __float_as_int(v));
+  else
+    atomicMin(reinterpret_cast<unsigned int *>(addr), __float_as_uint(v));
+}
+
+// kMaxLogit: also the largest content logit scale*<q_i,k_j> over every row and
+// visible key of each (sequence, head), into Params::max_logit (atomic max).
+template <int D, int BN, int NH, bool kPacked, bool kMaxLogit>
 __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -665,6 +687,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       const int h = t.h0 + w;
       const int i = t.m0 + r;                        // query position
       float m_run = -INFINITY;                       // running max, log2 units
+      float row_max = -INFINITY;                     // exact row maximum, log2 units
       float l_run = 0.f;                             // running denominator
       for (int j = 0; j < t.n_tiles; ++j) {
         const int g = jg + j;
@@ -695,7 +718,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
           }
         }
         if (!softmax_tile<D, BN>(lane_base, s_col, o_col, j, g, sl2, lo, hi, cls_mask, cls_none,
-                                 m_run, l_run, &pv_done[w], ctx)) {
+                                 m_run, l_run, row_max, &pv_done[w], ctx)) {
           ok = false;
           break;
         }
@@ -773,6 +796,14 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       if (p.lse != nullptr && i < t.len)
         p.lse[(packed ? t.row0 : static_cast<int64_t>(t.b) * p.lse_sb) + static_cast<int64_t>(h) * p.lse_sh +
               i] = lse_val;
+      if constexpr (kMaxLogit) {
+        // the unit's largest logit (log2 units back to natural): warp
+        // maximum, then one atomic per warp
+        float v = (i < t.len) ? row_max * kLn2 : -INFINITY;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        if ((r & 31) == 0 && v > -INFINITY) atomic_max_float(&p.max_logit[static_cast<int64_t>(t.b) * p.ml_sb + h], v);
+      }
     }
     // stores must have read shared memory before the CTA leaves
     if (r == 0) tma_store_wait_all();
@@ -782,7 +813,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   }
 }
 
-template <int D, int BN, int NH, bool kPacked>
+template <int D, int BN, int NH, bool kPacked, bool kMaxLogit = false>
 cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
   using C = Cfg<D, BN, NH>;
   alignas(64) CUtensorMap mq, mk, mv, mo;
@@ -813,7 +844,13 @@ cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
   p.out = static_cast<__nv_bfloat16 *>(a.out);
   p.o_sr = a.o_s[1];
   p.o_sh = a.o_s[2];
-  auto kern = fwd_tc_kernel<D, BN, NH, kPacked>;
+  p.max_logit = a.max_logit;
+  p.ml_sb = a.ml_sb;
+  if (kMaxLogit) {
+    // every entry starts at -inf; the kernel's units raise it
+    if ((e = launch_max_logit_init(a.max_logit, a.ml_sb, a.B, a.Hq, stream)) != cudaSuccess) return e;
+  }
+  auto kern = fwd_tc_kernel<D, BN, NH, kPacked, kMaxLogit>;
   static bool attr_set[64] = {};  // once per device (per instantiation)
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -836,20 +873,32 @@ cudaError_t launch(const FwdArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
+cudaError_t launch_max_logit_init(float *ml, int64_t sb, int B, int Hq, cudaStream_t stream) {
+  const int n = B * Hq;
+  if (n <= 0) return cudaSuccess;
+  max_logit_init_kernel<<<(n + 255) / 256, 256, 0, stream>>>(ml, sb, B, Hq);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream) {
   // Two query heads per CTA when they share a kv head (even group size) and
   // their S and O fit TMEM together; otherwise one.
   const bool pair = (a.Hq / a.Hkv) % 2 == 0;
   const bool packed = a.cu_seqlens != nullptr;
+  const bool ml = a.max_logit != nullptr;   // (batched inputs only)
+  if (packed && ml) return cudaErrorInvalidValue;
   switch (a.D) {
     case 64:
       if (packed) return pair ? launch<64, 128, 2, true>(a, stream) : launch<64, 64, 1, true>(a, stream);
+      if (ml) return pair ? launch<64, 128, 2, false, true>(a, stream) : launch<64, 64, 1, false, true>(a, stream);
       return pair ? launch<64, 128, 2, false>(a, stream) : launch<64, 64, 1, false>(a, stream);
     case 128:
       if (packed) return pair ? launch<128, 128, 2, true>(a, stream) : launch<128, 64, 1, true>(a, stream);
+      if (ml) return pair ? launch<128, 128, 2, false, true>(a, stream) : launch<128, 64, 1, false, true>(a, stream);
       return pair ? launch<128, 128, 2, false>(a, stream) : launch<128, 64, 1, false>(a, stream);
     case 256:
-      return packed ? launch<256, 64, 1, true>(a, stream) : launch<256, 64, 1, false>(a, stream);
+      if (packed) return launch<256, 64, 1, true>(a, stream);
+      return ml ? launch<256, 64, 1, false, true>(a, stream) : launch<256, 64, 1, false>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }

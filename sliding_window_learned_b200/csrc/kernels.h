@@ -26,6 +26,10 @@ struct FwdArgs {
   // head stride).  Null: the [B, L] batch above.
   const int *cu_seqlens = nullptr;
   int T = 0;
+  // Largest content logit per (batch, query head): [B, Hq] f32 (row stride
+  // ml_sb), batched inputs only; null: not computed.
+  float *max_logit = nullptr;
+  int64_t ml_sb = 0;
 };
 
 // Decode: q/out [B,Hq,D], caches [B,Smax,Hkv,D] (bf16), seqlens [B] int32
@@ -59,6 +63,8 @@ size_t decode_workspace_bytes(const DecodeArgs &a);
 int decode_max_splits_per_seq(const DecodeArgs &a);
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream);
+// Sets every entry of a [B, Hq] max-logit output to -inf.
+cudaError_t launch_max_logit_init(float *ml, int64_t sb, int B, int Hq, cudaStream_t stream);
 cudaError_t launch_fwd_cudacore(const FwdArgs &a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t stream);
 
