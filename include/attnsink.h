@@ -91,9 +91,9 @@ int attn_sink_fwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
  * attn_sink_fwd that also returns the largest pre-softmax logit of every
  * (batch, query head): max over rows i and visible keys j of
  * scale * <q_i, k_j>, the sink excluded (page "Dao-AILab/flash-attention"
- * contributor guide, task for issue #2986: expose the maximum pre-softmax
- * logit, per-head maxima of shape (batch, nheads), from the running row
- * maxima the kernel already keeps).
+ * contributor guide, the task for issue #2986: users want the largest logit
+ * before the softmax for monitoring, one value per batch and head, taken from
+ * the row maxima the kernel computes anyway).
  *
  *   max_logit  [B, Hq] f32 (innermost stride 1), written completely: -inf
  *              where a (batch, head) has no position (L = 0).

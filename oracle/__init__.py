@@ -138,7 +138,7 @@ def max_logit(q, k, window: int, scale: float):
     """The largest pre-softmax logit of every (batch, query head): the maximum
     over rows i and visible keys j in [max(0, i-W+1), i] of scale * <q_i, k_j>
     (kv head h // (Hq/Hkv)), the sink excluded (the flash-attention contributor
-    guide's task for issue #2986: per-head maxima of shape (batch, nheads)).
+    guide's task for issue #2986: one largest logit per batch and head).
     q [B,L,Hq,D], k [B,L,Hkv,D] as uint16 bf16 bits.  Returns [B, Hq] float64
     (-inf where L = 0).  Plain fp64, one key offset of the window at a time."""
     q, k = _u16(q), _u16(k)
