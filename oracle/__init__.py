@@ -134,6 +134,53 @@ def fwd_varlen(q, k, v, cu_seqlens, sinks, window: int, scale: float):
     return out, lse
 
 
+def _torch_forward(qd, kd, vd, sinks, window: int, scale: float):
+    """The forward as differentiable torch float64 operations: the window
+    mask, one sink column per head joined to the softmax and dropped after it
+    (page 1: the sink is a logit in the denominator with no value row).
+    qd [B,L,Hq,D], kd/vd [B,L,Hkv,D], sinks [Hq]; returns (O [B,L,Hq,D],
+    LSE [B,Hq,L])."""
+    import torch
+    B, L, Hq, D = qd.shape
+    Hkv = kd.shape[2]
+    kk = kd.repeat_interleave(Hq // Hkv, dim=2)
+    vv = vd.repeat_interleave(Hq // Hkv, dim=2)
+    # the scale is the float32 value the device receives, widened exactly
+    s = float(np.float32(scale)) * torch.einsum("bihd,bjhd->bhij", qd, kk)
+    i = torch.arange(L).view(L, 1)
+    j = torch.arange(L).view(1, L)
+    visible = (j <= i) & (j >= i - int(window) + 1)
+    s = s.masked_fill(~visible, float("-inf"))
+    full = torch.cat([s, sinks.view(1, Hq, 1, 1).expand(B, Hq, L, 1)], dim=-1)
+    lse = torch.logsumexp(full, dim=-1)
+    p = torch.exp(full - lse.unsqueeze(-1))[..., :L]
+    o = torch.einsum("bhij,bjhd->bihd", p, vv)
+    return o, lse
+
+
+def bwd(q, k, v, sinks, dout, window: int, scale: float):
+    """Gradients of the forward: for the loss sum(dout * O), the gradients
+    with respect to q, k, v and the sinks, by float64 automatic
+    differentiation of ``_torch_forward`` (the definition; page 4 names the
+    sink gradient, issue #2969, as computed from the unrounded O).
+    q [B,L,Hq,D], k/v [B,L,Hkv,D], dout [B,L,Hq,D] as uint16 bf16 bits,
+    sinks [Hq] float32 (finite or -inf).
+    Returns (dq, dk, dv, dsinks, O, LSE) float64 numpy arrays."""
+    import torch
+    q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
+    qd = torch.from_numpy(_bits_to_f64(q)).requires_grad_()
+    kd = torch.from_numpy(_bits_to_f64(k)).requires_grad_()
+    vd = torch.from_numpy(_bits_to_f64(v)).requires_grad_()
+    sd = torch.from_numpy(np.asarray(sinks, dtype=np.float32).astype(np.float64)).requires_grad_()
+    do = torch.from_numpy(_bits_to_f64(dout))
+    o, lse = _torch_forward(qd, kd, vd, sd, window, scale)
+    (o * do).sum().backward()
+    ds = sd.grad if sd.grad is not None else torch.zeros_like(sd)
+    ds = torch.nan_to_num(ds, nan=0.0)          # an -inf sink has no gradient
+    return (qd.grad.numpy(), kd.grad.numpy(), vd.grad.numpy(), ds.numpy(),
+            o.detach().numpy(), lse.detach().numpy())
+
+
 def max_logit(q, k, window: int, scale: float):
     """The largest pre-softmax logit of every (batch, query head): the maximum
     over rows i and visible keys j in [max(0, i-W+1), i] of scale * <q_i, k_j>
