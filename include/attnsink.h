@@ -144,6 +144,37 @@ int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k,
                            attn_tensor *lse, void *stream);
 
 /*
+ * Backward pass of attn_sink_fwd for the loss sum(dout * O): dq, dk, dv and
+ * the sinks' gradient (page "Dao-AILab/flash-attention" contributor guide:
+ * the FA4 backward's dK/dV and dQ phases, and issue #2969 on forming the
+ * sink's gradient from the unrounded O).  With P_ij = exp(s_ij - LSE_i),
+ * P_sink,i = exp(sink_h - LSE_i) and Dsum_i = dout_i . O_i:
+ *   dv_j = sum_i P_ij dout_i;  dS_ij = P_ij (dout_i . v_j - Dsum_i);
+ *   dq_i = scale sum_j dS_ij k_j;  dk_j = scale sum_i dS_ij q_i;
+ *   dsink_h = -sum_{b,i} P_sink,i Dsum_i.
+ *
+ *   q, dout     [B, L, Hq, D]  bf16
+ *   k, v        [B, L, Hkv, D] bf16
+ *   o           [B, L, Hq, D]  the forward's output: bf16 (as attn_sink_fwd
+ *               writes it; Dsum then carries its rounding) or f32 (Dsum exact,
+ *               the form issue #2969 asks for)
+ *   lse         [B, Hq, L]     f32, the forward's log-sum-exp (sink included)
+ *   sinks, window, scale: as for attn_sink_fwd.
+ *   dq          [B, L, Hq, D]  bf16, written completely
+ *   dk, dv      [B, L, Hkv, D] bf16, written completely (summed over the
+ *               query heads of each kv head)
+ *   dsink       [Hq] f32, summed over the batch
+ * D in {64, 128}.  Workspace: an fp32 dq accumulator and the row sums,
+ * B*L*Hq*(D+1)*4 bytes, from the library's stream-ordered pool.  Runs on
+ * warp-level (mma.sync) bf16 tensor-core products with fp32 accumulation; P
+ * and dS are rounded to bf16 for the products.
+ */
+int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
+                  const attn_tensor *o, const attn_tensor *lse, const attn_tensor *dout,
+                  const attn_tensor *sinks, int32_t window, float scale, attn_tensor *dq,
+                  attn_tensor *dk, attn_tensor *dv, attn_tensor *dsink, void *stream);
+
+/*
  * Single-token split-KV decode over a contiguous KV cache (page
  * "flashmla-optimization/docs/PATCH_STACK.md", section 3 "exact small-split
  * combine"; split-KV decode benchmark on the flash-attention contributor

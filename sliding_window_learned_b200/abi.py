@@ -34,7 +34,7 @@ _DTYPES = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float32: ATTN_DTYPE_F32,
            torch.int32: ATTN_DTYPE_I32, torch.float8_e4m3fn: ATTN_DTYPE_E4M3}
 
 # Every symbol include/attnsink.h declares.
-EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_max_logit", "attn_sink_fwd_varlen", "attn_sink_fwd_cudacore", "attn_sink_decode",
+EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_max_logit", "attn_sink_fwd_varlen", "attn_sink_bwd", "attn_sink_fwd_cudacore", "attn_sink_decode",
            "attn_sink_decode_chunked", "attn_sink_decode_paged", "attn_sink_decode_fp8",
            "attn_sink_decode_noalloc",
            "attn_sink_get_status",
@@ -70,6 +70,8 @@ def load() -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.argtypes = [P, P, P, P, i32, f32, P, P, V]
             fn.restype = ctypes.c_int
+        lib.attn_sink_bwd.argtypes = [P, P, P, P, P, P, P, i32, f32, P, P, P, P, V]
+        lib.attn_sink_bwd.restype = ctypes.c_int
         lib.attn_sink_fwd_max_logit.argtypes = [P, P, P, P, i32, f32, P, P, P, V]
         lib.attn_sink_fwd_max_logit.restype = ctypes.c_int
         lib.attn_sink_fwd_varlen.argtypes = [P, P, P, P, i32, P, i32, f32, P, P, V]
@@ -149,6 +151,18 @@ def attn_sink_fwd(q, k, v, sinks, window: int, scale: float, out, lse=None, stre
     rc = lib.attn_sink_fwd(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), int(window),
                            float(scale), _ref(ds[4]), _ref(ds[5]), _stream(stream, q))
     _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_bwd(q, k, v, o, lse, dout, sinks, window: int, scale: float, dq, dk, dv, dsink,
+                  stream=None):
+    """C ``attn_sink_bwd``: gradients of sum(dout * O) into dq, dk, dv (bf16)
+    and dsink ([Hq] f32); ``o`` is the forward's output (bf16 or f32)."""
+    lib = load()
+    ds = [describe(x) for x in (q, k, v, o, lse, dout, sinks, dq, dk, dv, dsink)]
+    rc = lib.attn_sink_bwd(_ref(ds[0]), _ref(ds[1]), _ref(ds[2]), _ref(ds[3]), _ref(ds[4]), _ref(ds[5]),
+                           _ref(ds[6]), int(window), float(scale), _ref(ds[7]), _ref(ds[8]), _ref(ds[9]),
+                           _ref(ds[10]), _stream(stream, q))
+    _check(rc, "attn_sink_bwd")
 
 
 def attn_sink_fwd_max_logit(q, k, v, sinks, window: int, scale: float, out, lse, max_logit,

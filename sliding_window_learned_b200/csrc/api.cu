@@ -419,6 +419,75 @@ int prep_decode(const attn_tensor *q, const attn_tensor *kcache, const attn_tens
   return ATTN_OK;
 }
 
+// Validates the backward's arguments and fills `a`.
+int prep_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v, const attn_tensor *o,
+             const attn_tensor *lse, const attn_tensor *dout, const attn_tensor *sinks, int32_t window,
+             float scale, attn_tensor *dq, attn_tensor *dk, attn_tensor *dv, attn_tensor *dsink, BwdArgs *a) {
+  int rc;
+  if ((rc = check_tensor(q, "q", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(k, "k", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(v, "v", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(dout, "dout", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if (!o || (o->dtype != ATTN_DTYPE_BF16 && o->dtype != ATTN_DTYPE_F32))
+    return fail(ATTN_EINVAL, "o: dtype must be bf16 or f32");
+  if ((rc = check_tensor(o, "o", o->dtype, 4, false))) return rc;
+  if ((rc = check_tensor(lse, "lse", ATTN_DTYPE_F32, 3, false))) return rc;
+  if ((rc = check_tensor(sinks, "sinks", ATTN_DTYPE_F32, 1, false))) return rc;
+  if ((rc = check_tensor(dq, "dq", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(dk, "dk", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(dv, "dv", ATTN_DTYPE_BF16, 4, true))) return rc;
+  if ((rc = check_tensor(dsink, "dsink", ATTN_DTYPE_F32, 1, false))) return rc;
+  const int64_t B = q->shape[0], L = q->shape[1], Hq = q->shape[2], D = q->shape[3], Hkv = k->shape[2];
+  for (int d = 0; d < 4; ++d) {
+    if (o->shape[d] != q->shape[d] || dout->shape[d] != q->shape[d] || dq->shape[d] != q->shape[d])
+      return fail(ATTN_EINVAL, "o, dout and dq must have q's shape");
+    if (v->shape[d] != k->shape[d] || dk->shape[d] != k->shape[d] || dv->shape[d] != k->shape[d])
+      return fail(ATTN_EINVAL, "v, dk and dv must have k's shape");
+  }
+  if (k->shape[0] != B || k->shape[1] != L || k->shape[3] != D) return fail(ATTN_EINVAL, "k shape does not match q");
+  if (lse->shape[0] != B || lse->shape[1] != Hq || lse->shape[2] != L) return fail(ATTN_EINVAL, "lse must be [B, Hq, L]");
+  if (sinks->shape[0] != Hq || dsink->shape[0] != Hq) return fail(ATTN_EINVAL, "sinks and dsink must have Hq entries");
+  if ((Hq > 1 && (sinks->stride[0] != 1 || dsink->stride[0] != 1)))
+    return fail(ATTN_EINVAL, "sinks and dsink must be contiguous");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(ATTN_EINVAL, "Hq must be a positive multiple of Hkv");
+  if (window < 1) return fail(ATTN_EINVAL, "window must be >= 1");
+  if (!finite_pos(scale)) return fail(ATTN_EINVAL, "scale must be finite and > 0");
+  if (D != 64 && D != 128) return fail(ATTN_EUNSUPPORTED, "backward: head dim %lld not supported (64, 128)", (long long)D);
+  if (B > 65535 || Hkv > 65535 || L > (1LL << 28)) return fail(ATTN_EUNSUPPORTED, "B, Hkv or L too large");
+  a->q = q->data;
+  a->k = k->data;
+  a->v = v->data;
+  a->o = o->data;
+  a->dout = dout->data;
+  a->lse = static_cast<const float *>(lse->data);
+  a->sinks = static_cast<const float *>(sinks->data);
+  a->dq = dq->data;
+  a->dk = dk->data;
+  a->dv = dv->data;
+  a->dsink = static_cast<float *>(dsink->data);
+  a->B = static_cast<int>(B);
+  a->L = static_cast<int>(L);
+  a->Hq = static_cast<int>(Hq);
+  a->Hkv = static_cast<int>(Hkv);
+  a->D = static_cast<int>(D);
+  a->W = window;
+  a->scale = scale;
+  a->o_f32 = o->dtype == ATTN_DTYPE_F32;
+  for (int d = 0; d < 3; ++d) {
+    a->q_s[d] = q->stride[d];
+    a->k_s[d] = k->stride[d];
+    a->v_s[d] = v->stride[d];
+    a->o_s[d] = o->stride[d];
+    a->do_s[d] = dout->stride[d];
+    a->dq_s[d] = dq->stride[d];
+    a->dk_s[d] = dk->stride[d];
+    a->dv_s[d] = dv->stride[d];
+  }
+  a->lse_s[0] = lse->stride[0];
+  a->lse_s[1] = lse->stride[1];
+  return ATTN_OK;
+}
+
 // Validates the paged-cache decode arguments and fills `out_args` (kc/vc are
 // the page pools, Smax = pages per sequence * page size); `*empty` as above.
 int prep_decode_paged(const attn_tensor *q, const attn_tensor *kpages, const attn_tensor *vpages,
@@ -697,6 +766,31 @@ int attn_sink_decode_fp8(const attn_tensor *q, const attn_tensor *kcache, const 
   const cudaError_t ef = cudaFreeAsync(ws, st);
   if (e != cudaSuccess) return fail_cuda(e, "attn_sink_decode_fp8 launch");
   if (ef != cudaSuccess) return fail_cuda(ef, "decode workspace release");
+  return ATTN_OK;
+}
+
+int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v, const attn_tensor *o,
+                  const attn_tensor *lse, const attn_tensor *dout, const attn_tensor *sinks, int32_t window,
+                  float scale, attn_tensor *dq, attn_tensor *dk, attn_tensor *dv, attn_tensor *dsink,
+                  void *stream) {
+  t_last_error[0] = '\0';
+  BwdArgs a;
+  int rc = prep_bwd(q, k, v, o, lse, dout, sinks, window, scale, dq, dk, dv, dsink, &a);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a.B == 0 || a.L == 0) {
+    const cudaError_t e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.Hq, st);
+    return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "attn_sink_bwd");
+  }
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  void *ws = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bwd_workspace_bytes(a), pool, st);
+  if (e != cudaSuccess) return fail_cuda(e, "backward workspace allocation");
+  e = launch_bwd(a, ws, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e != cudaSuccess) return fail_cuda(e, "attn_sink_bwd launch");
+  if (ef != cudaSuccess) return fail_cuda(ef, "backward workspace release");
   return ATTN_OK;
 }
 

@@ -56,6 +56,21 @@ struct DecodeArgs {
   const float *k_descale = nullptr, *v_descale = nullptr;
 };
 
+// Backward: q/dq/dout/o [B,L,Hq,D], k/v/dk/dv [B,L,Hkv,D] (bf16; o bf16 or
+// f32), lse [B,Hq,L] f32 from the forward, sinks [Hq] f32, dsink [Hq] f32.
+struct BwdArgs {
+  const void *q, *k, *v, *o, *dout;
+  const float *lse, *sinks;
+  void *dq, *dk, *dv;
+  float *dsink;
+  int B, L, Hq, Hkv, D, W;
+  float scale;
+  bool o_f32;
+  int64_t q_s[3], k_s[3], v_s[3], o_s[3], do_s[3], dq_s[3], dk_s[3], dv_s[3], lse_s[2];
+};
+size_t bwd_workspace_bytes(const BwdArgs &a);
+cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream);
+
 // Bytes of stream-ordered workspace one decode call needs (256-byte aligned
 // sections: plan, partial LSEs, partial outputs).
 size_t decode_workspace_bytes(const DecodeArgs &a);

@@ -1,0 +1,112 @@
+"""GPU parity of the backward pass (attn_sink_bwd) against the fp64 oracle.
+
+Bar (derived from the arithmetic: bf16 inputs, P and dS rounded to bf16 for
+the tensor-core products, fp32 accumulation): for each of dq, dk, dv,
+max|d| <= 2e-2 * max(1, max|ref|); for dsink, |d| <= 2e-2 * max(1, |ref|) per
+head; no NaN/Inf.  The forward's O enters either as f32 (the oracle's, so
+that dO . O is exact: the form issue #2969 asks for) or as the bf16 output of
+attn_sink_fwd with its LSE (the pipeline a trainer runs)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_learned_b200 as swl
+from sliding_window_learned_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+REL = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from sliding_window_learned_b200 import build
+    build.build()
+    oracle.build()
+
+
+def _case(B, L, Hq, Hkv, D, seed, sinks="uniform"):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, L, Hq, D, generator=g).bfloat16()
+    k = torch.randn(B, L, Hkv, D, generator=g).bfloat16()
+    v = torch.randn(B, L, Hkv, D, generator=g).bfloat16()
+    do = torch.randn(B, L, Hq, D, generator=g).bfloat16()
+    if sinks == "uniform":
+        s = torch.rand(Hq, generator=g) * 12.0 - 4.0
+    elif sinks == "none":
+        s = torch.full((Hq,), float("-inf"))
+    else:
+        s = torch.full((Hq,), float(sinks))
+    return q, k, v, do, s
+
+
+def _gpu_bwd(q, k, v, o, lse, do, s, W, scale):
+    dq = torch.full_like(q, float("nan"), device=DEV)
+    dk = torch.full_like(k, float("nan"), device=DEV)
+    dv = torch.full_like(v, float("nan"), device=DEV)
+    dsink = torch.full((q.shape[2],), float("nan"), device=DEV)
+    swl.attn_sink_bwd(q.to(DEV), k.to(DEV), v.to(DEV), o.to(DEV), lse.to(DEV), do.to(DEV), s.to(DEV), W,
+                      scale, dq, dk, dv, dsink)
+    torch.cuda.synchronize()
+    assert swl.attn_sink_get_status() == 0
+    return [t.float().cpu().numpy() for t in (dq, dk, dv, dsink)]
+
+
+def _check(got, ref, what):
+    for name, g, r in zip(("dq", "dk", "dv"), got[:3], ref[:3]):
+        assert np.isfinite(g).all(), f"{what}: non-finite {name}"
+        err = float(np.abs(g - r).max())
+        assert err <= REL * max(1.0, float(np.abs(r).max())), f"{what}: {name} max|d| = {err}"
+    assert np.isfinite(got[3]).all(), f"{what}: non-finite dsink"
+    err = np.abs(got[3] - ref[3])
+    assert (err <= REL * np.maximum(1.0, np.abs(ref[3]))).all(), f"{what}: dsink |d| = {err.max()}"
+
+
+CASES = [  # B, L, Hq, Hkv, D, W, sinks
+    (1, 256, 4, 2, 64, 64, "uniform"),
+    (2, 300, 8, 2, 128, 513, "uniform"),
+    (1, 200, 4, 4, 64, 1, "uniform"),
+    (1, 517, 6, 2, 128, 1 << 30, "uniform"),
+    (2, 129, 4, 1, 128, 33, "none"),
+    (1, 190, 4, 2, 128, 100, 20.0),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}L{c[1]}Hq{c[2]}Hkv{c[3]}D{c[4]}W{c[5]}s{c[6]}" for c in CASES])
+@pytest.mark.parametrize("o_kind", ["f32", "bf16"])
+def test_bwd_against_oracle(case, o_kind):
+    B, L, Hq, Hkv, D, W, sk = case
+    q, k, v, do, s = _case(B, L, Hq, Hkv, D, seed=L + D + W % 89, sinks=sk)
+    scale = 1.0 / np.sqrt(D)
+    ref = oracle.bwd(inputs.bits(q), inputs.bits(k), inputs.bits(v), s.numpy(), inputs.bits(do), W, scale)
+    if o_kind == "f32":
+        o = torch.from_numpy(ref[4]).float()
+        lse = torch.from_numpy(ref[5]).float()
+    else:
+        o, lse = swl.fwd(q.to(DEV), k.to(DEV), v.to(DEV), s.to(DEV), W, scale)
+    got = _gpu_bwd(q, k, v, o, lse, do, s, W, scale)
+    _check(got, ref, f"bwd ({o_kind} O)")
+    if sk == "none":
+        assert (got[3] == 0).all()
+    elif o_kind == "f32":
+        # with the unrounded O, dO . O is exact and so is the sink gradient's
+        # sum (fp32): the precision issue #2969 is about does not arise
+        err = np.abs(got[3] - ref[3])
+        assert (err <= 1e-4 * np.maximum(1e-3, np.abs(ref[3]))).all(), f"dsink rel err {err.max()}"
+
+
+def test_bwd_prefill_heads_sampled():
+    """The prefill workload's shape at a quarter of its length (B2 Hq32 Hkv4
+    L1024 D128 W513) through attn_sink_fwd then attn_sink_bwd: every gradient
+    finite; the first kv group (8 query heads) against the oracle."""
+    B, L, Hq, Hkv, D, W = 2, 1024, 32, 4, 128, 513
+    q, k, v, do, s = _case(B, L, Hq, Hkv, D, seed=21)
+    scale = 1.0 / np.sqrt(D)
+    o, lse = swl.fwd(q.to(DEV), k.to(DEV), v.to(DEV), s.to(DEV), W, scale)
+    got = _gpu_bwd(q, k, v, o, lse, do, s, W, scale)
+    for g in got:
+        assert np.isfinite(g).all()
+    ref = oracle.bwd(inputs.bits(q[:, :, :8]), inputs.bits(k[:, :, :1]), inputs.bits(v[:, :, :1]),
+                     s[:8].numpy(), inputs.bits(do[:, :, :8]), W, scale)
+    _check([got[0][:, :, :8], got[1][:, :, :1], got[2][:, :, :1], got[3][:8]], ref, "prefill heads")
