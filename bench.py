@@ -11,9 +11,10 @@ ranks, from CUDA events around each prefill launch; the decode figure (HBM
 GB/s of algorithmic bytes) is reported beside it, and after the timed steps
 the same decode over a paged copy of its cache (256-position pages at random
 pool positions, attn_sink_decode_paged) is timed as `decode_paged`, the decode
-over the cache quantised to e4m3 (attn_sink_decode_fp8) as `decode_fp8`, and the
+over the cache quantised to e4m3 (attn_sink_decode_fp8) as `decode_fp8`, the
 forward over a seeded mix of 24 packed sequences (attn_sink_fwd_varlen) as
-`fwd_varlen`.
+`fwd_varlen`, and the backward pass on the prefill workload (attn_sink_bwd) as
+`bwd`.
 `--impl reference` times
 the fp64 CPU oracle on a bounded sample of the same prefill workload.
 
@@ -331,12 +332,39 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device status error in the packed forward")
     del vq, vk, vv, vout, vlse
 
+    # ---- the backward pass on the prefill workload: O and LSE from the
+    # forward above, a seeded N(0, 1) upstream gradient ----
+    bw_gen = torch.Generator(device=dev).manual_seed(2000 + rank)
+    bdo = torch.randn(q.shape, device=dev, generator=bw_gen).bfloat16()
+    bdq, bdk, bdv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bds = torch.empty(pcfg.Hq, dtype=torch.float32, device=dev)
+    fwd()
+
+    def bwd():
+        swl.attn_sink_bwd(q, k, v, out, lse, bdo, sinks, pcfg.W, pcfg.scale, bdq, bdk, bdv, bds, stream)
+
+    Kb = max(3, min(K, 30))
+    for _ in range(3):
+        bwd()
+    torch.cuda.synchronize()
+    t_bwd = 0.0
+    for _ in range(Kb):
+        flush.fill_(1.0)
+        e0.record(stream)
+        bwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_bwd += e0.elapsed_time(e1) / 1e3
+    if swl.attn_sink_get_status() != 0:
+        raise RuntimeError("device status error in the backward pass")
+    del bdo, bdq, bdk, bdv
+
     # ---- max over ranks ----
-    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8], dtype=torch.float64,
+    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8, t_bwd], dtype=torch.float64,
                          device=dev)
     if world > 1:
         dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8 = times.tolist()
+    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8, t_bwd = times.tolist()
 
     if rank != 0:
         return
@@ -395,6 +423,12 @@ def run_ours(args, rank, world, local_rank):
                        "frac": round(vl_flops / (t_varlen / Kv) / 1e12 / bf16_peak, 4),
                        "what": "attn_sink_fwd_varlen on 24 packed sequences of U[1, 4096] tokens "
                                f"(T = {vl_T}), Hq32 Hkv4 D128 W513, L2 flushed before each call"},
+        "bwd": {"value": round(world * Kb * 2.5 * fwd_flops / t_bwd / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_call": round(t_bwd / Kb * 1e3, 5),
+                "frac": round(2.5 * fwd_flops / (t_bwd / Kb) / 1e12 / bf16_peak, 4),
+                "what": "attn_sink_bwd (dq, dk, dv, dsink) on the prefill workload, O and LSE from "
+                        "attn_sink_fwd; useful FLOPs = 10 D per visible pair (2.5x the forward's), "
+                        "L2 flushed before each call"},
         "e2e": {"value": round(world * Ke * fwd_flops / t_e2e / 1e12, 4), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "attn_sink_fwd with pinned host inputs copied in and O, LSE copied out each step"},
