@@ -323,15 +323,21 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(strides_el[2]) * eb,
                                  static_cast<cuuint64_t>(strides_el[1]) * eb,
                                  static_cast<cuuint64_t>(strides_el[0]) * eb};
-  // 128 bytes of the innermost dimension per box row (the swizzle span)
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, static_cast<cuuint32_t>(box_rows), 1};
+  // 128 bytes of the innermost dimension per box row (the swizzle span); an
+  // f32 map instead spans the whole row, unswizzled
+  const bool f32 = elem_bytes == 4;
+  if (f32 && (d0 > 256 || (d0 * 4) % 16 != 0)) return cudaErrorInvalidValue;
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(f32 ? d0 : 128 / elem_bytes), 1,
+                             static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   alignas(64) CUtensorMap map;
-  const CUresult r = encode(&map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                            4, const_cast<void *>(base), dims,
-                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : f32         ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUresult r = encode(&map, dt, 4, const_cast<void *>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            f32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   memcpy(map_out, &map, sizeof(CUtensorMap));
   std::lock_guard<std::mutex> lk(g_tma_mu);
@@ -485,7 +491,7 @@ int prep_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v, c
   }
   a->lse_s[0] = lse->stride[0];
   a->lse_s[1] = lse->stride[1];
-  return ATTN_OK;
+  return status_ptr(&a->status);
 }
 
 // Validates the paged-cache decode arguments and fills `out_args` (kc/vc are

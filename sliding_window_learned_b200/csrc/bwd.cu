@@ -301,6 +301,8 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_main_kernel(const BwdParams p
 }
 
 // ------------------------------------------------------------------ dQ out
+// fp32 [B, L, H, D] accumulator -> strided bf16 (dQ; dK and dV after the
+// tensor-core main pass)
 __global__ void bwd_dq_kernel(const float *acc, __nv_bfloat16 *dq, int B, int L, int Hq, int D, int64_t s0,
                               int64_t s1, int64_t s2) {
   const int64_t n = static_cast<int64_t>(B) * L * Hq * D;
@@ -356,19 +358,32 @@ cudaError_t launch_main(const BwdArgs &a, float *dq_acc, const float *dsum, cuda
 
 }  // namespace
 
+// Workspace: the fp32 dQ accumulator [B, L, Hq, D], Dsum [B, Hq, L], and for
+// D = 128 (the tensor-core main pass) fp32 dK, dV accumulators [B, L, Hkv, D].
+namespace {
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
+}  // namespace
+
 size_t bwd_workspace_bytes(const BwdArgs &a) {
   const size_t acc = sizeof(float) * static_cast<size_t>(a.B) * a.L * a.Hq * a.D;
   const size_t ds = sizeof(float) * static_cast<size_t>(a.B) * a.Hq * a.L;
-  return (acc + 255) / 256 * 256 + (ds + 255) / 256 * 256;
+  const size_t kv = a.D == 128 ? 2 * align256(sizeof(float) * static_cast<size_t>(a.B) * a.L * a.Hkv * a.D) : 0;
+  return align256(acc) + align256(ds) + kv;
 }
 
 cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   float *dq_acc = reinterpret_cast<float *>(ws);
   const size_t acc_bytes = sizeof(float) * static_cast<size_t>(a.B) * a.L * a.Hq * a.D;
-  float *dsum = reinterpret_cast<float *>(ws + (acc_bytes + 255) / 256 * 256);
+  float *dsum = reinterpret_cast<float *>(ws + align256(acc_bytes));
+  const size_t ds_bytes = sizeof(float) * static_cast<size_t>(a.B) * a.Hq * a.L;
+  const size_t kv_bytes = sizeof(float) * static_cast<size_t>(a.B) * a.L * a.Hkv * a.D;
+  float *dk_acc = reinterpret_cast<float *>(ws + align256(acc_bytes) + align256(ds_bytes));
+  float *dv_acc = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(dk_acc) + align256(kv_bytes));
+  const bool tc = a.D == 128;
   cudaError_t e = cudaMemsetAsync(dq_acc, 0, acc_bytes, stream);
   if (e != cudaSuccess) return e;
+  if (tc && (e = cudaMemsetAsync(dk_acc, 0, align256(kv_bytes) + kv_bytes, stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.Hq, stream)) != cudaSuccess) return e;
   dim3 rg((a.L + 63) / 64, a.Hq, a.B);
   if (a.o_f32)
@@ -384,15 +399,23 @@ cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   switch (a.D) {
     case 64: e = launch_main<64>(a, dq_acc, dsum, stream); break;
-    case 128: e = launch_main<128>(a, dq_acc, dsum, stream); break;
+    case 128: e = launch_bwd_main_tc(a, dsum, dq_acc, dk_acc, dv_acc, stream); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  const int64_t n = static_cast<int64_t>(a.B) * a.L * a.Hq * a.D;
-  const int blocks = static_cast<int>(n / 256 + 1 < 148 * 16 ? n / 256 + 1 : 148 * 16);
-  bwd_dq_kernel<<<blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16 *>(a.dq), a.B, a.L, a.Hq, a.D,
-                                            a.dq_s[0], a.dq_s[1], a.dq_s[2]);
-  return cudaGetLastError();
+  auto convert = [&](const float *acc, void *out, int H, const int64_t *s) {
+    const int64_t n = static_cast<int64_t>(a.B) * a.L * H * a.D;
+    const int blocks = static_cast<int>(n / 256 + 1 < 148 * 16 ? n / 256 + 1 : 148 * 16);
+    bwd_dq_kernel<<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(out), a.B, a.L, H, a.D, s[0],
+                                              s[1], s[2]);
+    return cudaGetLastError();
+  };
+  if ((e = convert(dq_acc, a.dq, a.Hq, a.dq_s)) != cudaSuccess) return e;
+  if (tc) {
+    if ((e = convert(dk_acc, a.dk, a.Hkv, a.dk_s)) != cudaSuccess) return e;
+    if ((e = convert(dv_acc, a.dv, a.Hkv, a.dv_s)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace attnsink

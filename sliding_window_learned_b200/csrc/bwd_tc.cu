@@ -1,0 +1,641 @@
+// bwd_tc.cu -- backward pass of sliding-window attention with a learned
+// per-head sink on the 5th-generation tensor cores (tcgen05, TMEM, TMA), head
+// dimension 128.  The gradients are those of bwd.cu (page "Dao-AILab/
+// flash-attention" contributor guide: the FA4 backward kernels and issue
+// #2969):
+//   P_ij = exp(s_ij - LSE_i), Dsum_i = dO_i . O_i,
+//   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . v_j - Dsum_i),
+//   dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j.
+// Dsum and the sink gradient come from bwd.cu's row kernel.
+//
+// A work unit is one block of 128 keys of one kv head (the TMEM lanes) and a
+// slice of the query heads that share it; its steps walk those heads and
+// every 64-query block that sees a key of the block.  Per step, five products
+// with fp32 accumulators in TMEM:
+//   S^T  = K Q^T      [128 keys x 64 queries]   A = K (smem), B = Q (smem)
+//   dP^T = V dO^T     [128 x 64]                A = V, B = dO
+//   dV  += P^T dO     [128 keys x 128]          A = P^T (bf16, TMEM), B = dO (smem, N-major)
+//   dK  += dS^T Q     [128 x 128]               A = dS^T (bf16, TMEM), B = Q (smem, N-major)
+//   dQ^T = K^T dS^T   [128 channels x 64]       A = K (smem, M-major), B = dS^T (smem, N-major)
+// All five have M = 128 (keys or channels on the TMEM lanes); dQ is formed
+// transposed so that it needs no 64-row accumulator.  P^T and dS^T live in
+// their own TMEM columns, so the next step's S^T and dP^T are computed while
+// this step's exponentials are taken.  TMEM columns (512):
+//   S^T 0..63 | dP^T 64..127 | P^T 128..159, dS^T 160..191 (bf16 pairs) |
+//   dV 192..319 | dK 320..447 | dQ^T 448..511
+//
+// Warp roles (384 threads, one CTA per SM, persistent over units):
+//   warps 0-3  one thread per key row: P^T, dS^T from S^T, dP^T, LSE, Dsum
+//   warps 4-7  one thread per channel: dQ^T out of TMEM into a shared f32
+//              [64 queries x 128] tile, added into the fp32 dQ workspace by
+//              one TMA bulk reduction per step; at a unit's end dK, dV (rows)
+//   warp 8     producer: K, V per unit, Q, dO per step (TMA, a ring of
+//              kStages slots) and the step's LSE and Dsum rows
+//   warp 9     TMEM allocation and the MMA issue (one thread)
+//   warps 10-11 idle (they pad the third warpgroup, which hands registers
+//              to the first)
+// dK and dV are summed over the units of a kv head in fp32 workspaces
+// (atomic adds), converted to bf16 afterwards like dQ.  Every wait is
+// bounded; a timeout records ATTN_ETIMEOUT and every role returns.
+#include <cuda.h>
+#include <math.h>
+
+#include <type_traits>
+
+#include "kernels.h"
+#include "ptx.cuh"
+#include "status.cuh"
+
+namespace attnsink {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kBK = 128;                        // keys per unit (TMEM lanes)
+constexpr int kBQ = 64;                         // queries per step
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr uint32_t kTmemThreads = 288;          // warps 0-7 and the MMA warp
+// Registers after reallocation: P^T/dS^T warpgroup, drain warpgroup (kept at
+// the launch value), producer/MMA warpgroup.
+constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8, kRegsSoftmax = 200, kRegsDrain = kRegsLaunch,
+                   kRegsOther = 136;
+static_assert(128 * (kRegsSoftmax + kRegsDrain + kRegsOther) <= kRegsLaunch * kThreads,
+              "register split exceeds the launch allocation");
+constexpr uint32_t kBarTmem = 1, kBarDrain = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDS = 160, kColDV = 192, kColDK = 320,
+                   kColDQ = 448, kTmemCols = 512;
+
+// Pipeline depths: Q/dO ring slots (the producer runs kStages - 1 steps
+// ahead), K/V buffers (2: the next unit's K, V load during this unit).
+constexpr int kStages = 3, kKVBuf = 1;
+
+// shared memory, from a 1024-byte aligned base (128-byte swizzled tiles)
+constexpr int kKVTile = kBK * kD * 2;           // a K or V tile: two 64-channel chunks of 128 rows
+constexpr int kQTile = kBQ * kD * 2;            // a Q or dO tile: two chunks of 64 rows
+constexpr int kDSTile = kBK * kBQ * 2;          // dS^T: 128 key rows of 64 queries
+constexpr int kOffK = 0;                        // [kKVBuf] K tiles (units alternate)
+constexpr int kOffV = kOffK + kKVBuf * kKVTile; // [kKVBuf] V tiles
+constexpr int kOffQ = kOffV + kKVBuf * kKVTile; // [kStages] Q tiles (ring slots)
+constexpr int kOffDO = kOffQ + kStages * kQTile;      // [kStages] dO tiles
+constexpr int kOffDS = kOffDO + kStages * kQTile;     // [2] dS^T tiles (steps alternate)
+constexpr int kOffRow = kOffDS + 2 * kDSTile;   // [kStages][LSE*log2e x 64, Dsum x 64] f32
+constexpr int kOffStage = kOffRow + kStages * 2 * kBQ * 4;   // dQ tile [64 queries][128] f32
+constexpr int kOffBar = kOffStage + kBQ * kD * 4;
+static_assert(kOffStage % 128 == 0, "bulk-copy staging alignment");
+constexpr int kBarBytes = 256;
+constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared-memory budget");
+
+enum : int { kWhereKv = 201, kWhereFull = 202, kWhereEmpty = 203, kWhereS = 204, kWhereP = 205,
+             kWhereDq = 206, kWhereDkv = 207 };
+
+struct Params {
+  const float *lse, *dsum;
+  float *dq_acc, *dk_acc, *dv_acc;
+  int *status;
+  int B, L, Hq, Hkv, W, G, hsplit, nkb, num_units;
+  float scale, sl2;                     // scale, scale * log2(e)
+  int64_t lse_sb, lse_sh;
+};
+
+// Unit u: key block kb (slowest: the earliest blocks see the most queries
+// under a causal window, so they start first), head slice hs, kv head hk,
+// batch b.  Its steps are (head h0 + s / nq, query block q_lo + s % nq).
+struct Unit {
+  int j0, hk, b, h0, nh, q_lo, nq;
+};
+
+__device__ __forceinline__ Unit unit_at(const Params &p, int u) {
+  Unit t;
+  const int per_kb = p.hsplit * p.Hkv * p.B;
+  const int kb = u / per_kb;
+  int r = u - kb * per_kb;
+  const int hs = r % p.hsplit;
+  r /= p.hsplit;
+  t.hk = r % p.Hkv;
+  t.b = r / p.Hkv;
+  t.j0 = kb * kBK;
+  t.nh = p.G / p.hsplit;
+  t.h0 = t.hk * p.G + hs * t.nh;
+  // queries that see a key of [j0, j0 + 127]: [j0, j0 + 127 + W - 1], clipped to L
+  const int last = min(p.L - 1, t.j0 + kBK - 1 + min(p.W - 1, p.L));
+  t.q_lo = t.j0 / kBQ;
+  t.nq = last / kBQ - t.q_lo + 1;
+  return t;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const WaitCtx &ctx, int where) {
+  const bool r = mbar_wait(bar, parity, ctx, where);
+  return __all_sync(0xffffffffu, r);
+}
+
+// Waits without looking at the abort flag, for draining in-flight copies on
+// the way out (bounded by the same limit).
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmDQ, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sK = smem + kOffK, *sV = smem + kOffV, *sQ = smem + kOffQ, *sDO = smem + kOffDO;
+  uint8_t *sDS = smem + kOffDS;
+  float *sRow = reinterpret_cast<float *>(smem + kOffRow);
+  uint64_t *kv_full = reinterpret_cast<uint64_t *>(smem + kOffBar);   // [kKVBuf] K, V of a unit landed
+  uint64_t *kv_empty = kv_full + kKVBuf; // [kKVBuf] a unit's last product read its K, V
+  uint64_t *full = kv_empty + kKVBuf;    // [kStages] a step's Q, dO (TMA) and rows (32 lanes) landed
+  uint64_t *empty = full + kStages;      // [kStages] a step's dV, dK products read its Q, dO
+  uint64_t *s_full = empty + kStages;    // S^T, dP^T of a step computed
+  uint64_t *s_free = s_full + 1;         // ... and read out of TMEM (128 arrivals)
+  uint64_t *p_full = s_free + 1;         // P^T, dS^T of a step in TMEM and dS^T in smem (128)
+  uint64_t *pbuf_free = p_full + 1;      // a step's dV, dK products read P^T, dS^T
+  uint64_t *dq_full = pbuf_free + 1;     // a step's dQ^T computed
+  uint64_t *dq_empty = dq_full + 1;      // ... and read out of TMEM (128)
+  uint64_t *dsm_free = dq_empty + 1;     // [2] a step's dQ^T product read its dS^T tile
+  uint64_t *dkv_full = dsm_free + 2;     // a unit's last dV, dK products finished
+  uint64_t *dkv_free = dkv_full + 1;     // ... and dK, dV read out of TMEM (128)
+  uint64_t *mma_done = dkv_free + 1;     // every product of the CTA finished
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  const WaitCtx ctx{abort_flag, p.status};
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kKVBuf; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 32);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(&dsm_free[i], 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(pbuf_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(dkv_full, 1);
+    mbar_init(dkv_free, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // TMEM: the MMA warp allocates all 512 columns (one CTA per SM); the TMEM
+  // warps read the base after one named barrier of exactly those warps.
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  uint32_t tmem = 0;
+  const bool tmem_warp = warp < 8 || warp == kMmaWarp;
+  if (tmem_warp) {
+    tc_fence_before();
+    named_barrier_sync(kBarTmem, kTmemThreads);
+    tc_fence_after();
+    tmem = *tmem_slot;
+  }
+  if (warp >= 8) {
+  // Producer/MMA warpgroup (the idle padding warps included): hand registers
+  // to the P^T/dS^T warpgroup.
+  setmaxnreg_dec<kRegsOther>();
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+    }
+    bool ok = true;
+    int g = 0, ul = 0;
+    int kv_issued = 0;                        // units whose K, V copies were issued
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
+      const Unit t = unit_at(p, u);
+      const int kvb = ul % kKVBuf;
+      if (lane == 0) {
+        // the buffer's previous unit has finished with its K and V
+        if (ul >= kKVBuf &&
+            !mbar_wait(&kv_empty[kvb], static_cast<uint32_t>(ul / kKVBuf - 1) & 1u, ctx, kWhereKv))
+          ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&kv_full[kvb], 2 * kKVTile);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_4d(sK + kvb * kKVTile + c * kBK * 128, &tmK, &kv_full[kvb], c * 64, t.hk, t.j0, t.b);
+            tma_load_4d(sV + kvb * kKVTile + c * kBK * 128, &tmV, &kv_full[kvb], c * 64, t.hk, t.j0, t.b);
+          }
+          kv_issued = ul + 1;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int steps = t.nh * t.nq;
+      for (int s = 0; ok && s < steps; ++s) {
+        const int slot = g % kStages;
+        const int h = t.h0 + s / t.nq;
+        const int i0 = (t.q_lo + s % t.nq) * kBQ;
+        // the step's rows, fetched while the slot drains: LSE in log2 units
+        // (+inf past the end, so P = 0) and Dsum
+        float lr[kBQ / 32], dr[kBQ / 32];
+#pragma unroll
+        for (int e = 0; e < kBQ / 32; ++e) {
+          const int i = i0 + lane + 32 * e;
+          const bool in = i < p.L;
+          lr[e] = in ? p.lse[t.b * p.lse_sb + h * p.lse_sh + i] * kLog2e : INFINITY;
+          dr[e] = in ? p.dsum[(static_cast<int64_t>(t.b) * p.Hq + h) * p.L + i] : 0.f;
+        }
+        if (lane == 0 && g >= kStages &&
+            !mbar_wait(&empty[slot], static_cast<uint32_t>(g / kStages - 1) & 1u, ctx, kWhereEmpty))
+          ok = false;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        float *row = sRow + slot * 2 * kBQ;
+#pragma unroll
+        for (int e = 0; e < kBQ / 32; ++e) {
+          row[lane + 32 * e] = lr[e];
+          row[kBQ + lane + 32 * e] = dr[e];
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[slot], 2 * kQTile);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_4d(sQ + slot * kQTile + c * kBQ * 128, &tmQ, &full[slot], c * 64, h, i0, t.b);
+            tma_load_4d(sDO + slot * kQTile + c * kBQ * 128, &tmDO, &full[slot], c * 64, h, i0, t.b);
+          }
+        } else {
+          mbar_arrive(&full[slot]);
+        }
+        ++g;                                  // steps whose copies were issued
+      }
+    }
+    if (!ok && lane == 0) {
+      // Leaving early: let the copies already issued land before the CTA
+      // (and its shared memory) goes away.
+      for (int k = max(0, kv_issued - kKVBuf); k < kv_issued; ++k)
+        drain_wait(&kv_full[k % kKVBuf], static_cast<uint32_t>(k / kKVBuf) & 1u);
+      for (int k = max(0, g - kStages); k < g; ++k)
+        drain_wait(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc_bf16(kBK, kBQ, 0, 0);    // K-major A and B
+      constexpr uint32_t idesc_kv = umma_idesc_bf16(kBK, kD, 0, 1);    // A in TMEM, B N-major
+      constexpr uint32_t idesc_dq = umma_idesc_bf16(kD, kBQ, 1, 1);    // A M-major, B N-major
+      // 128-byte swizzle, 8-row groups 1024 bytes apart; the leading offset is
+      // the distance between 64-element chunks along M or N for the
+      // M/N-major operands (K-major operands ignore it)
+      const uint32_t hi = umma_desc_hi_sw128(1024);
+      const uint32_t k_lo = umma_desc_lo(smem_u32(sK), 16);
+      const uint32_t v_lo = umma_desc_lo(smem_u32(sV), 16);
+      const uint32_t q_lo = umma_desc_lo(smem_u32(sQ), 16);
+      const uint32_t do_lo = umma_desc_lo(smem_u32(sDO), 16);
+      const uint32_t qn_lo = umma_desc_lo(smem_u32(sQ), kBQ * 128);     // Q as an N-major B
+      const uint32_t don_lo = umma_desc_lo(smem_u32(sDO), kBQ * 128);   // dO as an N-major B
+      const uint32_t km_lo = umma_desc_lo(smem_u32(sK), kBK * 128);     // K as an M-major A
+      const uint32_t ds_lo = umma_desc_lo(smem_u32(sDS), kBK * 128);    // dS^T as an N-major B
+      bool ok = true;
+      struct Pending {
+        int g, slot, kvb, ul;
+        bool first, last;
+      };
+      Pending pend{0, 0, 0, 0, false, false};
+      bool have = false;
+      // the second half of a step: dV, dK once P^T, dS^T are in, then dQ^T
+      auto finish = [&](const Pending &r) -> bool {
+        if (!mbar_wait(p_full, static_cast<uint32_t>(r.g) & 1u, ctx, kWhereP)) return false;
+        // the first step of a unit overwrites dK, dV: the previous unit's
+        // must have been read out of TMEM
+        if (r.first && r.ul > 0 && !mbar_wait(dkv_free, static_cast<uint32_t>(r.ul - 1) & 1u, ctx, kWhereDkv))
+          return false;
+        tc_fence_after();
+        const uint32_t acc0 = r.first ? 0u : 1u;
+#pragma unroll
+        for (int kk = 0; kk < kBQ / 16; ++kk)
+          umma_ts_w(tmem + kColDV, tmem + kColP + kk * 8, don_lo + ((r.slot * kQTile + kk * 16 * 128) >> 4), hi,
+                    idesc_kv, kk > 0 ? 1u : acc0);
+#pragma unroll
+        for (int kk = 0; kk < kBQ / 16; ++kk)
+          umma_ts_w(tmem + kColDK, tmem + kColDS + kk * 8, qn_lo + ((r.slot * kQTile + kk * 16 * 128) >> 4), hi,
+                    idesc_kv, kk > 0 ? 1u : acc0);
+        umma_commit(pbuf_free);
+        umma_commit(&empty[r.slot]);
+        if (r.last) umma_commit(dkv_full);
+        // dQ^T overwrites the previous step's, which must have been read out
+        if (r.g > 0 && !mbar_wait(dq_empty, static_cast<uint32_t>(r.g - 1) & 1u, ctx, kWhereDq)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          umma_ss_w(tmem + kColDQ, km_lo + ((r.kvb * kKVTile + kk * 16 * 128) >> 4), hi,
+                    ds_lo + (((r.g & 1) * kDSTile + kk * 16 * 128) >> 4), hi, idesc_dq, kk > 0 ? 1u : 0u);
+        umma_commit(dq_full);
+        umma_commit(&dsm_free[r.g & 1]);
+        if (r.last) umma_commit(&kv_empty[r.kvb]);
+        return true;
+      };
+      int g = 0, ul = 0;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
+        const Unit t = unit_at(p, u);
+        const int kvb = ul % kKVBuf;
+        // with one K/V buffer the previous unit must let go of it first
+        if (kKVBuf == 1 && have) {
+          have = false;
+          if (!finish(pend)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!mbar_wait(&kv_full[kvb], static_cast<uint32_t>(ul / kKVBuf) & 1u, ctx, kWhereKv)) {
+          ok = false;
+          break;
+        }
+        const int steps = t.nh * t.nq;
+        for (int s = 0; s < steps; ++s, ++g) {
+          const int slot = g % kStages;
+          if (!mbar_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull)) {
+            ok = false;
+            break;
+          }
+          // S^T and dP^T overwrite the previous step's, which the softmax
+          // warps must have read out
+          if (g > 0 && !mbar_wait(s_free, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
+            const uint32_t ka = ((kvb * kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
+            const uint32_t qa = ((slot * kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
+            umma_ss_w(tmem + kColS, k_lo + ka, hi, q_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t ka = ((kvb * kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
+            const uint32_t qa = ((slot * kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
+            umma_ss_w(tmem + kColDP, v_lo + ka, hi, do_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full);
+          if (have && !finish(pend)) {
+            ok = false;
+            break;
+          }
+          pend = Pending{g, slot, kvb, ul, s == 0, s == steps - 1};
+          have = true;
+        }
+      }
+      if (ok && have) finish(pend);
+      // Every tensor-core operation of this CTA has finished before teardown.
+      umma_commit(mma_done);
+      drain_wait(mma_done, 0);
+    }
+    __syncwarp();
+  }
+  } else if (warp < 4) {
+    setmaxnreg_inc<kRegsSoftmax>();
+    // ----------------------------------- P^T, dS^T (one key row per thread)
+    const int r = threadIdx.x;                        // key row == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    bool ok = true;
+    int g = 0;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      const Unit t = unit_at(p, u);
+      const int j = t.j0 + r;                         // key position
+      const int steps = t.nh * t.nq;
+      for (int s = 0; s < steps; ++s, ++g) {
+        const int slot = g % kStages;
+        const int i0 = (t.q_lo + s % t.nq) * kBQ;
+        if (!warp_wait(s_full, static_cast<uint32_t>(g) & 1u, ctx, kWhereS) ||
+            !warp_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s0[32], s1[32], d0[32], d1[32];
+        tmem_ld32(lane_base + kColS, s0);
+        tmem_ld32(lane_base + kColS + 32, s1);
+        tmem_ld32(lane_base + kColDP, d0);
+        tmem_ld32(lane_base + kColDP + 32, d1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_free);                          // the next step's S^T, dP^T may start
+        // Does any (key, query) pair of the step fall outside the window or
+        // past the end of the sequence?  If so, this row's visible columns
+        // are [vlo, vhi] (query i = i0 + column sees key j iff
+        // j <= i < L and i - j < W).
+        const bool edge = (t.j0 + kBK - 1 > i0) || (t.j0 < i0 + kBQ - p.W) || (i0 + kBQ > p.L);
+        const int vlo = j - i0;
+        const int vhi = min(j - i0 + min(p.W - 1, p.L), p.L - 1 - i0);
+        const float4 *lse4 = reinterpret_cast<const float4 *>(sRow + slot * 2 * kBQ);
+        const float4 *dsum4 = lse4 + kBQ / 4;
+        uint32_t pp[32], dd[32];                      // bf16 pairs of P^T and dS^T
+        // one branch-free copy per case (a per-element branch inside the
+        // unrolled loop costs the unmasked steps as much as the masked ones)
+        auto half = [&](auto masked, const uint32_t (&sv)[32], const uint32_t (&dv)[32], int c0) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 l4 = lse4[(c0 + c) >> 2];
+            const float4 m4 = dsum4[(c0 + c) >> 2];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+            float pe[4], de[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              pe[e] = ex2_approx(__uint_as_float(sv[c + e]) * p.sl2 - lv[e]);
+              if constexpr (decltype(masked)::value) {
+                const int col = c0 + c + e;
+                pe[e] = (col >= vlo && col <= vhi) ? pe[e] : 0.f;
+              }
+              de[e] = pe[e] * (__uint_as_float(dv[c + e]) - mv[e]);
+            }
+            pp[(c0 + c) / 2] = pack_bf16x2(pe[0], pe[1]);
+            pp[(c0 + c) / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+            dd[(c0 + c) / 2] = pack_bf16x2(de[0], de[1]);
+            dd[(c0 + c) / 2 + 1] = pack_bf16x2(de[2], de[3]);
+          }
+        };
+        if (edge) {
+          half(std::true_type{}, s0, d0, 0);
+          half(std::true_type{}, s1, d1, 32);
+        } else {
+          half(std::false_type{}, s0, d0, 0);
+          half(std::false_type{}, s1, d1, 32);
+        }
+        // P^T, dS^T overwrite the previous step's (its dV, dK products must
+        // have read them); dS^T's shared tile was last read two steps ago
+        if ((g > 0 && !warp_wait(pbuf_free, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereP)) ||
+            (g >= 2 && !warp_wait(&dsm_free[g & 1], static_cast<uint32_t>((g >> 1) - 1) & 1u, ctx, kWhereDq))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(lane_base + kColP, pp);
+        tmem_st32(lane_base + kColDS, dd);
+        // dS^T row r: 64 queries = 128 bytes, 16-byte units swizzled by row
+        uint8_t *dsrow = sDS + (g & 1) * kDSTile + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4 *>(dsrow + ((q ^ (r & 7)) << 4)) =
+              make_uint4(dd[4 * q], dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
+        tmem_wait_st();
+        fence_proxy_async_smem();                     // dS^T visible to the tensor cores
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+    }
+  } else {
+    // ------------------------- dQ^T out of TMEM; dK, dV at the end of a unit
+    const int rr = (warp & 3) * 32 + lane;            // TMEM lane: channel (dQ^T), key row (dK, dV)
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    float *stage = reinterpret_cast<float *>(smem + kOffStage);
+    bool ok = true;
+    int g = 0, ul = 0;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
+      const Unit t = unit_at(p, u);
+      const int steps = t.nh * t.nq;
+      for (int s = 0; s < steps; ++s, ++g) {
+        const int h = t.h0 + s / t.nq;
+        const int i0 = (t.q_lo + s % t.nq) * kBQ;
+        if (!warp_wait(dq_full, static_cast<uint32_t>(g) & 1u, ctx, kWhereDq)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t x0[32], x1[32];
+        tmem_ld32(lane_base + kColDQ, x0);
+        tmem_ld32(lane_base + kColDQ + 32, x1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(dq_empty);                        // the next dQ^T may overwrite it
+        // the previous step's reduction has read the staging tile
+        if (rr == 0) tma_store_wait_read();
+        named_barrier_sync(kBarDrain, 128);
+        // dQ^T column -> dQ row-major tile: for each query the warp writes 32
+        // consecutive channels
+#pragma unroll
+        for (int c = 0; c < 32; ++c) stage[c * kD + rr] = __uint_as_float(x0[c]) * p.scale;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) stage[(32 + c) * kD + rr] = __uint_as_float(x1[c]) * p.scale;
+        fence_proxy_async_smem();
+        named_barrier_sync(kBarDrain, 128);
+        if (rr == 0) {
+          // rows past the end of the sequence are clipped by the unit
+          tma_reduce_add_4d(&tmDQ, stage, 0, h, i0, t.b);
+          tma_store_commit();
+        }
+        if (s == steps - 1) {
+          if (!warp_wait(dkv_full, static_cast<uint32_t>(ul) & 1u, ctx, kWhereDkv)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int j = t.j0 + rr;
+          const int64_t kv_row = ((static_cast<int64_t>(t.b) * p.L + j) * p.Hkv + t.hk) * kD;
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t k32[32], v32[32];
+            tmem_ld32(lane_base + kColDK + c * 32, k32);
+            tmem_ld32(lane_base + kColDV + c * 32, v32);
+            tmem_wait_ld();
+            if (j < p.L) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                atomicAdd(reinterpret_cast<float4 *>(p.dk_acc + kv_row + c * 32 + 4 * q),
+                          make_float4(__uint_as_float(k32[4 * q]) * p.scale, __uint_as_float(k32[4 * q + 1]) * p.scale,
+                                      __uint_as_float(k32[4 * q + 2]) * p.scale, __uint_as_float(k32[4 * q + 3]) * p.scale));
+                atomicAdd(reinterpret_cast<float4 *>(p.dv_acc + kv_row + c * 32 + 4 * q),
+                          make_float4(__uint_as_float(v32[4 * q]), __uint_as_float(v32[4 * q + 1]),
+                                      __uint_as_float(v32[4 * q + 2]), __uint_as_float(v32[4 * q + 3])));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(dkv_free);                      // the next unit's first dV, dK may overwrite them
+        }
+      }
+    }
+    // the reductions must have read shared memory before the CTA leaves
+    if (rr == 0) tma_store_wait_all();
+  }
+  // ---- teardown: every TMEM user is done before the allocator frees it ----
+  if (tmem_warp) {
+    tc_fence_before();
+    named_barrier_sync(kBarTmem, kTmemThreads);
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float *dk_acc, float *dv_acc,
+                               cudaStream_t stream) {
+  if (a.D != kD) return cudaErrorInvalidValue;
+  alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
+  cudaError_t e;
+  if ((e = make_tma_bshd(&mq, a.q, a.B, a.L, a.Hq, kD, a.q_s, kBQ)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mk, a.k, a.B, a.L, a.Hkv, kD, a.k_s, kBK)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mv, a.v, a.B, a.L, a.Hkv, kD, a.v_s, kBK)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mdo, a.dout, a.B, a.L, a.Hq, kD, a.do_s, kBQ)) != cudaSuccess) return e;
+  const int64_t acc_s[3] = {static_cast<int64_t>(a.L) * a.Hq * kD, static_cast<int64_t>(a.Hq) * kD, kD};
+  if ((e = make_tma_bshd(&mdq, dq_acc, a.B, a.L, a.Hq, kD, acc_s, kBQ, 4)) != cudaSuccess) return e;
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  static int sm_count[64] = {};
+  if (dev >= 0 && dev < 64 && sm_count[dev] == 0)
+    if ((e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+  const int sms = (dev >= 0 && dev < 64) ? sm_count[dev] : 148;
+  Params p;
+  p.lse = a.lse;
+  p.dsum = dsum;
+  p.dq_acc = dq_acc;
+  p.dk_acc = dk_acc;
+  p.dv_acc = dv_acc;
+  p.status = a.status;
+  p.B = a.B;
+  p.L = a.L;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.W = a.W;
+  p.G = a.Hq / a.Hkv;
+  p.nkb = (a.L + kBK - 1) / kBK;
+  // Split each kv head's query heads over units until there are about four
+  // units per SM (whole heads per unit; the units of a kv head add their dK,
+  // dV into the same fp32 rows).
+  const int64_t base = static_cast<int64_t>(p.nkb) * a.Hkv * a.B;
+  p.hsplit = 1;
+  for (int hs = 1; hs <= p.G; ++hs) {
+    if (p.G % hs) continue;
+    p.hsplit = hs;
+    if (base * hs >= 4LL * sms) break;
+  }
+  const int64_t units = base * p.hsplit;
+  if (units > (1LL << 30)) return cudaErrorInvalidValue;
+  p.num_units = static_cast<int>(units);
+  p.scale = a.scale;
+  p.sl2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
+  p.lse_sb = a.lse_s[0];
+  p.lse_sh = a.lse_s[1];
+  if ((e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)) !=
+      cudaSuccess)
+    return e;
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  bwd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace attnsink

@@ -67,9 +67,15 @@ struct BwdArgs {
   float scale;
   bool o_f32;
   int64_t q_s[3], k_s[3], v_s[3], o_s[3], do_s[3], dq_s[3], dk_s[3], dv_s[3], lse_s[2];
+  int *status;                             // device status word (2 ints)
 };
 size_t bwd_workspace_bytes(const BwdArgs &a);
 cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream);
+// The tcgen05 main pass of the backward for D = 128: dQ, dK, dV summed in
+// fp32 workspaces ([B, L, Hq, D], [B, L, Hkv, D], zeroed by the caller) from
+// Dsum ([B, Hq, L]).
+cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float *dk_acc, float *dv_acc,
+                               cudaStream_t stream);
 
 // Bytes of stream-ordered workspace one decode call needs (256-byte aligned
 // sections: plan, partial LSEs, partial outputs).
@@ -89,6 +95,8 @@ cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t str
 // Returns cudaErrorInvalidValue if the driver rejects the description.
 // elem_bytes = 1 describes a byte tensor (FP8) instead, with a box of
 // {128, 1, box_rows, 1}: 128 one-byte elements per 128-byte swizzled row.
+// elem_bytes = 4 describes an f32 tensor with whole rows per box
+// ({d0, 1, box_rows, 1}, d0 <= 256, no swizzle), for bulk reductions.
 cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
                           int64_t d0, const int64_t strides_el[3], int box_rows, int elem_bytes = 2);
 
