@@ -23,6 +23,8 @@
 // workspace by atomic adds and converted to bf16 by the third launch.
 #include <math.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -68,37 +70,78 @@ struct BwdParams {
 
 // ------------------------------------------------------------------ rows
 // Dsum[b, h, i] = dO . O for every row, and dsink[h] -= exp(sink - LSE) * Dsum
-// (one atomic per block).  One warp per row, 8 rows per warp in turn.
-template <typename OT>
+// (one atomic per block).  A block takes 64 rows of one (batch, head); each
+// warp takes 8 of them with every load issued before the first sum, each lane
+// D/32 consecutive channels (vector loads when the rows are aligned).
+template <int E, bool kVec, typename T>
+__device__ __forceinline__ void load_row(const T *p, float (&v)[E]) {
+  if constexpr (kVec && std::is_same<T, float>::value && E == 4) {
+    const float4 x = *reinterpret_cast<const float4 *>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else if constexpr (kVec && std::is_same<T, float>::value && E == 2) {
+    const float2 x = *reinterpret_cast<const float2 *>(p);
+    v[0] = x.x; v[1] = x.y;
+  } else if constexpr (kVec && !std::is_same<T, float>::value && E == 4) {
+    const uint2 x = *reinterpret_cast<const uint2 *>(p);
+    v[0] = __uint_as_float(x.x << 16); v[1] = __uint_as_float(x.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(x.y << 16); v[3] = __uint_as_float(x.y & 0xFFFF0000u);
+  } else if constexpr (kVec && !std::is_same<T, float>::value && E == 2) {
+    const uint32_t x = *reinterpret_cast<const uint32_t *>(p);
+    v[0] = __uint_as_float(x << 16); v[1] = __uint_as_float(x & 0xFFFF0000u);
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = static_cast<float>(p[e]);
+  }
+}
+
+template <typename OT, int D, bool kVec>
 __global__ void __launch_bounds__(256) bwd_rows_kernel(const OT *o, const __nv_bfloat16 *dout,
                                                        const float *lse, const float *sinks, float *dsum,
-                                                       float *dsink, int L, int Hq, int D, int64_t o_sb,
+                                                       float *dsink, int L, int Hq, int64_t o_sb,
                                                        int64_t o_sl, int64_t o_sh, int64_t d_sb, int64_t d_sl,
                                                        int64_t d_sh, int64_t lse_sb, int64_t lse_sh) {
+  constexpr int E = D / 32;
   const int h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i0 = blockIdx.x * 64 + warp;             // rows i0, i0 + 8, ..., i0 + 56
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int i = i0 + 8 * k;
+    float a = 0.f;
+    if (i < L) {
+      float ov[E], dv[E];
+      load_row<E, kVec>(o + b * o_sb + i * o_sl + h * o_sh + lane * E, ov);
+      load_row<E, kVec>(dout + b * d_sb + i * d_sl + h * d_sh + lane * E, dv);
+#pragma unroll
+      for (int e = 0; e < E; ++e) a += ov[e] * dv[e];
+    }
+    acc[k] = a;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], off);
+  // lane k < 8 finishes row i0 + 8k
+  float mine = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mine = (lane == k) ? acc[k] : mine;
+  const int i = i0 + 8 * lane;
   const float sink = sinks[h];
   float part = 0.f;
-  for (int i = blockIdx.x * 64 + warp; i < min(L, blockIdx.x * 64 + 64); i += 8) {
-    const OT *orow = o + b * o_sb + i * o_sl + h * o_sh;
-    const __nv_bfloat16 *drow = dout + b * d_sb + i * d_sl + h * d_sh;
-    float acc = 0.f;
-    for (int d = lane; d < D; d += 32) acc += static_cast<float>(orow[d]) * __bfloat162float(drow[d]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      dsum[(static_cast<int64_t>(b) * Hq + h) * L + i] = acc;
-      const float l = lse[b * lse_sb + h * lse_sh + i];
-      if (sink != -INFINITY) part -= __expf(sink - l) * acc;
-    }
+  if (lane < 8 && i < L) {
+    dsum[(static_cast<int64_t>(b) * Hq + h) * L + i] = mine;
+    if (sink != -INFINITY) part = -__expf(sink - lse[b * lse_sb + h * lse_sh + i]) * mine;
   }
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
   __shared__ float red[8];
   if (lane == 0) red[warp] = part;
   __syncthreads();
   if (threadIdx.x == 0) {
-    float s = 0.f;
-    for (int w = 0; w < 8; ++w) s += red[w];
-    if (s != 0.f) atomicAdd(&dsink[h], s);
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    if (t != 0.f) atomicAdd(&dsink[h], t);
   }
 }
 
@@ -302,19 +345,26 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_main_kernel(const BwdParams p
 
 // ------------------------------------------------------------------ dQ out
 // fp32 [B, L, H, D] accumulator -> strided bf16 (dQ; dK and dV after the
-// tensor-core main pass)
-__global__ void bwd_dq_kernel(const float *acc, __nv_bfloat16 *dq, int B, int L, int Hq, int D, int64_t s0,
-                              int64_t s1, int64_t s2) {
-  const int64_t n = static_cast<int64_t>(B) * L * Hq * D;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int d = static_cast<int>(e % D);
-    const int64_t r = e / D;
-    const int h = static_cast<int>(r % Hq);
-    const int64_t r2 = r / Hq;
-    const int i = static_cast<int>(r2 % L);
-    const int b = static_cast<int>(r2 / L);
-    dq[b * s0 + i * s1 + h * s2 + d] = __float2bfloat16_rn(acc[e]);
+// tensor-core main pass): one thread per 8 channels, two 16-byte loads and
+// one 16-byte store.
+template <int D>
+__global__ void bwd_convert_kernel(const float *acc, __nv_bfloat16 *out, uint32_t rows, uint32_t H, uint32_t L,
+                                   int64_t s0, int64_t s1, int64_t s2) {
+  constexpr uint32_t kPer = D / 8;
+  const uint64_t n = static_cast<uint64_t>(rows) * kPer;
+  for (uint64_t e = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t r = static_cast<uint32_t>(e / kPer), c = static_cast<uint32_t>(e % kPer) * 8;
+    const uint32_t h = r % H, bi = r / H;
+    const uint32_t i = bi % L, b = bi / L;
+    const float4 x = *reinterpret_cast<const float4 *>(acc + static_cast<uint64_t>(r) * D + c);
+    const float4 y = *reinterpret_cast<const float4 *>(acc + static_cast<uint64_t>(r) * D + c + 4);
+    uint4 v;
+    v.x = pack_bf16x2(x.x, x.y);
+    v.y = pack_bf16x2(x.z, x.w);
+    v.z = pack_bf16x2(y.x, y.y);
+    v.w = pack_bf16x2(y.z, y.w);
+    *reinterpret_cast<uint4 *>(out + b * s0 + i * s1 + h * s2 + c) = v;
   }
 }
 
@@ -386,16 +436,29 @@ cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
   if (tc && (e = cudaMemsetAsync(dk_acc, 0, align256(kv_bytes) + kv_bytes, stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.Hq, stream)) != cudaSuccess) return e;
   dim3 rg((a.L + 63) / 64, a.Hq, a.B);
-  if (a.o_f32)
-    bwd_rows_kernel<float><<<rg, 256, 0, stream>>>(
-        static_cast<const float *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.sinks, dsum,
-        a.dsink, a.L, a.Hq, a.D, a.o_s[0], a.o_s[1], a.o_s[2], a.do_s[0], a.do_s[1], a.do_s[2], a.lse_s[0],
-        a.lse_s[1]);
-  else
-    bwd_rows_kernel<__nv_bfloat16><<<rg, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.sinks,
-        dsum, a.dsink, a.L, a.Hq, a.D, a.o_s[0], a.o_s[1], a.o_s[2], a.do_s[0], a.do_s[1], a.do_s[2],
-        a.lse_s[0], a.lse_s[1]);
+  // vector loads of O need its rows aligned to the per-lane chunk (bf16 rows
+  // are: their strides and base are 16-byte multiples)
+  const int E = a.D / 32;
+  const int eb = a.o_f32 ? 4 : 2;
+  const bool ovec = reinterpret_cast<uintptr_t>(a.o) % (E * eb) == 0 && a.o_s[0] % E == 0 && a.o_s[1] % E == 0 &&
+                    a.o_s[2] % E == 0;
+  auto rows = [&](auto ot, auto dconst, auto vec) {
+    using OT = decltype(ot);
+    bwd_rows_kernel<OT, decltype(dconst)::value, decltype(vec)::value><<<rg, 256, 0, stream>>>(
+        static_cast<const OT *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.sinks, dsum, a.dsink,
+        a.L, a.Hq, a.o_s[0], a.o_s[1], a.o_s[2], a.do_s[0], a.do_s[1], a.do_s[2], a.lse_s[0], a.lse_s[1]);
+  };
+  using D64 = std::integral_constant<int, 64>;
+  using D128 = std::integral_constant<int, 128>;
+  using VY = std::true_type;
+  using VN = std::false_type;
+  if (a.D == 128) {
+    if (a.o_f32) { if (ovec) rows(float{}, D128{}, VY{}); else rows(float{}, D128{}, VN{}); }
+    else rows(__nv_bfloat16{}, D128{}, VY{});
+  } else {
+    if (a.o_f32) { if (ovec) rows(float{}, D64{}, VY{}); else rows(float{}, D64{}, VN{}); }
+    else rows(__nv_bfloat16{}, D64{}, VY{});
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   switch (a.D) {
     case 64: e = launch_main<64>(a, dq_acc, dsum, stream); break;
@@ -404,10 +467,16 @@ cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
   }
   if (e != cudaSuccess) return e;
   auto convert = [&](const float *acc, void *out, int H, const int64_t *s) {
-    const int64_t n = static_cast<int64_t>(a.B) * a.L * H * a.D;
-    const int blocks = static_cast<int>(n / 256 + 1 < 148 * 16 ? n / 256 + 1 : 148 * 16);
-    bwd_dq_kernel<<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(out), a.B, a.L, H, a.D, s[0],
-                                              s[1], s[2]);
+    const uint64_t rows64 = static_cast<uint64_t>(a.B) * a.L * H;
+    if (rows64 > 0xFFFFFFFFull) return cudaErrorInvalidValue;
+    const uint64_t n = rows64 * (a.D / 8);
+    const int blocks = static_cast<int>(n / 256 + 1 < 148 * 8 ? n / 256 + 1 : 148 * 8);
+    if (a.D == 128)
+      bwd_convert_kernel<128><<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(out),
+                                                          static_cast<uint32_t>(rows64), H, a.L, s[0], s[1], s[2]);
+    else
+      bwd_convert_kernel<64><<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(out),
+                                                         static_cast<uint32_t>(rows64), H, a.L, s[0], s[1], s[2]);
     return cudaGetLastError();
   };
   if ((e = convert(dq_acc, a.dq, a.Hq, a.dq_s)) != cudaSuccess) return e;
