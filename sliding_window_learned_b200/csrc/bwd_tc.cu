@@ -24,16 +24,16 @@
 //   S^T 0..63 | dP^T 64..127 | P^T 128..159, dS^T 160..191 (bf16 pairs) |
 //   dV 192..319 | dK 320..447 | dQ^T 448..511
 //
-// Warp roles (384 threads, one CTA per SM, persistent over units):
-//   warps 0-3  one thread per key row: P^T, dS^T from S^T, dP^T, LSE, Dsum
-//   warps 4-7  one thread per channel: dQ^T out of TMEM into a shared f32
+// Warp roles (512 threads, one CTA per SM, persistent over units):
+//   warps 0-7  one thread per key row and half of the step's queries (two
+//              warpgroups): P^T, dS^T from S^T, dP^T, LSE, Dsum
+//   warps 8-11 one thread per channel: dQ^T out of TMEM into a shared f32
 //              [64 queries x 128] tile, added into the fp32 dQ workspace by
 //              one TMA bulk reduction per step; at a unit's end dK, dV (rows)
-//   warp 8     producer: K, V per unit, Q, dO per step (TMA, a ring of
+//   warp 12    producer: K, V per unit, Q, dO per step (TMA, a ring of
 //              kStages slots) and the step's LSE and Dsum rows
-//   warp 9     TMEM allocation and the MMA issue (one thread)
-//   warps 10-11 idle (they pad the third warpgroup, which hands registers
-//              to the first)
+//   warp 13    TMEM allocation and the MMA issue (one thread)
+//   warps 14-15 idle (they pad the fourth warpgroup)
 // dK and dV are summed over the units of a kv head in fp32 workspaces
 // (atomic adds), converted to bf16 afterwards like dQ.  Every wait is
 // bounded; a timeout records ATTN_ETIMEOUT and every role returns.
@@ -52,14 +52,14 @@ namespace {
 constexpr int kD = 128;
 constexpr int kBK = 128;                        // keys per unit (TMEM lanes)
 constexpr int kBQ = 64;                         // queries per step
-constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr uint32_t kTmemThreads = 288;          // warps 0-7 and the MMA warp
-// Registers after reallocation: P^T/dS^T warpgroup, drain warpgroup (kept at
-// the launch value), producer/MMA warpgroup.
-constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8, kRegsSoftmax = 200, kRegsDrain = kRegsLaunch,
-                   kRegsOther = 136;
-static_assert(128 * (kRegsSoftmax + kRegsDrain + kRegsOther) <= kRegsLaunch * kThreads,
+constexpr int kThreads = 512;
+constexpr int kProducerWarp = 12, kMmaWarp = 13;
+constexpr uint32_t kTmemThreads = 416;          // warps 0-11 and the MMA warp
+// Registers after reallocation: the two P^T/dS^T warpgroups hand some to the
+// producer/MMA warpgroup; the drain warpgroup keeps the launch value.
+constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8, kRegsSoftmax = 120, kRegsDrain = kRegsLaunch,
+                   kRegsOther = 144;
+static_assert(128 * (2 * kRegsSoftmax + kRegsDrain + kRegsOther) <= kRegsLaunch * kThreads,
               "register split exceeds the launch allocation");
 constexpr uint32_t kBarTmem = 1, kBarDrain = 2;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *full = kv_empty + kKVBuf;    // [kStages] a step's Q, dO (TMA) and rows (32 lanes) landed
   uint64_t *empty = full + kStages;      // [kStages] a step's dV, dK products read its Q, dO
   uint64_t *s_full = empty + kStages;    // S^T, dP^T of a step computed
-  uint64_t *s_free = s_full + 1;         // ... and read out of TMEM (128 arrivals)
-  uint64_t *p_full = s_free + 1;         // P^T, dS^T of a step in TMEM and dS^T in smem (128)
+  uint64_t *s_free = s_full + 1;         // ... and read out of TMEM (256 arrivals)
+  uint64_t *p_full = s_free + 1;         // P^T, dS^T of a step in TMEM and dS^T in smem (256)
   uint64_t *pbuf_free = p_full + 1;      // a step's dV, dK products read P^T, dS^T
   uint64_t *dq_full = pbuf_free + 1;     // a step's dQ^T computed
   uint64_t *dq_empty = dq_full + 1;      // ... and read out of TMEM (128)
@@ -182,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) mbar_init(&dsm_free[i], 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
+    mbar_init(s_free, 256);
+    mbar_init(p_full, 256);
     mbar_init(pbuf_free, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -201,17 +201,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   uint32_t tmem = 0;
-  const bool tmem_warp = warp < 8 || warp == kMmaWarp;
+  const bool tmem_warp = warp < 12 || warp == kMmaWarp;
   if (tmem_warp) {
     tc_fence_before();
     named_barrier_sync(kBarTmem, kTmemThreads);
     tc_fence_after();
     tmem = *tmem_slot;
   }
-  if (warp >= 8) {
-  // Producer/MMA warpgroup (the idle padding warps included): hand registers
-  // to the P^T/dS^T warpgroup.
-  setmaxnreg_dec<kRegsOther>();
+  if (warp >= 12) {
+  setmaxnreg_inc<kRegsOther>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -404,11 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  } else if (warp < 4) {
-    setmaxnreg_inc<kRegsSoftmax>();
-    // ----------------------------------- P^T, dS^T (one key row per thread)
-    const int r = threadIdx.x;                        // key row == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  } else if (warp < 8) {
+    // --------------- P^T, dS^T: one key row per thread, 32 query columns per
+    // warpgroup (warpgroup 0 the first half of the step's queries)
+    setmaxnreg_dec<kRegsSoftmax>();
+    const int r = threadIdx.x & 127;                  // key row == TMEM lane
+    const int c0 = (warp >> 2) * 32;                  // this warpgroup's first column
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = true;
     int g = 0;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
@@ -424,11 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t s0[32], s1[32], d0[32], d1[32];
-        tmem_ld32(lane_base + kColS, s0);
-        tmem_ld32(lane_base + kColS + 32, s1);
-        tmem_ld32(lane_base + kColDP, d0);
-        tmem_ld32(lane_base + kColDP + 32, d1);
+        uint32_t sv[32], dv[32];
+        tmem_ld32(lane_base + kColS + c0, sv);
+        tmem_ld32(lane_base + kColDP + c0, dv);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(s_free);                          // the next step's S^T, dP^T may start
@@ -439,16 +437,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool edge = (t.j0 + kBK - 1 > i0) || (t.j0 < i0 + kBQ - p.W) || (i0 + kBQ > p.L);
         const int vlo = j - i0;
         const int vhi = min(j - i0 + min(p.W - 1, p.L), p.L - 1 - i0);
-        const float4 *lse4 = reinterpret_cast<const float4 *>(sRow + slot * 2 * kBQ);
+        const float4 *lse4 = reinterpret_cast<const float4 *>(sRow + slot * 2 * kBQ + c0);
         const float4 *dsum4 = lse4 + kBQ / 4;
-        uint32_t pp[32], dd[32];                      // bf16 pairs of P^T and dS^T
+        uint32_t pp[16], dd[16];                      // bf16 pairs of P^T and dS^T
         // one branch-free copy per case (a per-element branch inside the
         // unrolled loop costs the unmasked steps as much as the masked ones)
-        auto half = [&](auto masked, const uint32_t (&sv)[32], const uint32_t (&dv)[32], int c0) {
+        auto cols = [&](auto masked) {
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
-            const float4 l4 = lse4[(c0 + c) >> 2];
-            const float4 m4 = dsum4[(c0 + c) >> 2];
+            const float4 l4 = lse4[c >> 2];
+            const float4 m4 = dsum4[c >> 2];
             const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
             const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
             float pe[4], de[4];
@@ -461,19 +459,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               de[e] = pe[e] * (__uint_as_float(dv[c + e]) - mv[e]);
             }
-            pp[(c0 + c) / 2] = pack_bf16x2(pe[0], pe[1]);
-            pp[(c0 + c) / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
-            dd[(c0 + c) / 2] = pack_bf16x2(de[0], de[1]);
-            dd[(c0 + c) / 2 + 1] = pack_bf16x2(de[2], de[3]);
+            pp[c / 2] = pack_bf16x2(pe[0], pe[1]);
+            pp[c / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+            dd[c / 2] = pack_bf16x2(de[0], de[1]);
+            dd[c / 2 + 1] = pack_bf16x2(de[2], de[3]);
           }
         };
-        if (edge) {
-          half(std::true_type{}, s0, d0, 0);
-          half(std::true_type{}, s1, d1, 32);
-        } else {
-          half(std::false_type{}, s0, d0, 0);
-          half(std::false_type{}, s1, d1, 32);
-        }
+        if (edge)
+          cols(std::true_type{});
+        else
+          cols(std::false_type{});
         // P^T, dS^T overwrite the previous step's (its dV, dK products must
         // have read them); dS^T's shared tile was last read two steps ago
         if ((g > 0 && !warp_wait(pbuf_free, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereP)) ||
@@ -482,13 +477,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        tmem_st32(lane_base + kColP, pp);
-        tmem_st32(lane_base + kColDS, dd);
-        // dS^T row r: 64 queries = 128 bytes, 16-byte units swizzled by row
+        tmem_st16(lane_base + kColP + c0 / 2, pp);
+        tmem_st16(lane_base + kColDS + c0 / 2, dd);
+        // dS^T row r: 64 queries = 128 bytes, 16-byte units swizzled by row;
+        // this warpgroup's 32 queries are units c0/8 .. c0/8 + 3
         uint8_t *dsrow = sDS + (g & 1) * kDSTile + r * 128;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4 *>(dsrow + ((q ^ (r & 7)) << 4)) =
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4 *>(dsrow + (((c0 / 8 + q) ^ (r & 7)) << 4)) =
               make_uint4(dd[4 * q], dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
         tmem_wait_st();
         fence_proxy_async_smem();                     // dS^T visible to the tensor cores
