@@ -426,6 +426,9 @@ def run_ours(args, rank, world, local_rank):
         "bwd": {"value": round(world * Kb * 2.5 * fwd_flops / t_bwd / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_call": round(t_bwd / Kb * 1e3, 5),
                 "frac": round(2.5 * fwd_flops / (t_bwd / Kb) / 1e12 / bf16_peak, 4),
+                "traffic_main_pass": profiled_traffic("bwd_tc", ["sliding_window_learned_b200/csrc/bwd_tc.cu",
+                                                                 "sliding_window_learned_b200/csrc/bwd.cu",
+                                                                 "sliding_window_learned_b200/csrc/ptx.cuh"]),
                 "what": "attn_sink_bwd (dq, dk, dv, dsink) on the prefill workload, O and LSE from "
                         "attn_sink_fwd; useful FLOPs = 10 D per visible pair (2.5x the forward's), "
                         "L2 flushed before each call"},

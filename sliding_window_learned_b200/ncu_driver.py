@@ -3,6 +3,9 @@ captures (Nsight Compute) of a single kernel on a bounded device footprint.
 
   python -m sliding_window_learned_b200.ncu_driver --op fwd --workload prefill --launches 3
   python -m sliding_window_learned_b200.ncu_driver --op decode --workload decode-small --launches 3
+  python -m sliding_window_learned_b200.ncu_driver --op bwd --workload prefill --launches 2
+
+(--op bwd runs one forward for O and LSE, then the backward passes.)
 
 It prints no timings (numbers taken under a profiler are not measurements);
 it exits non-zero if the device reports an error.
@@ -30,7 +33,7 @@ WORKLOADS = {
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["fwd", "decode"], required=True)
+    ap.add_argument("--op", choices=["fwd", "decode", "bwd"], required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
     ap.add_argument("--launches", type=int, default=3)
     a = ap.parse_args(argv)
@@ -38,14 +41,24 @@ def main(argv=None) -> int:
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     cfg = WORKLOADS[a.workload]
-    if a.op == "fwd":
+    if a.op in ("fwd", "bwd"):
         if not isinstance(cfg, inputs.Prefill):
-            raise SystemExit("fwd needs a prefill workload")
+            raise SystemExit(f"{a.op} needs a prefill workload")
         x = inputs.make_prefill(cfg, seed=0, device=dev)
         out = torch.empty_like(x["q"])
         lse = torch.empty(cfg.B, cfg.Hq, cfg.L, dtype=torch.float32, device=dev)
-        for _ in range(a.launches):
+        if a.op == "fwd":
+            for _ in range(a.launches):
+                abi.attn_sink_fwd(x["q"], x["k"], x["v"], x["sinks"], cfg.W, cfg.scale, out, lse)
+        else:
             abi.attn_sink_fwd(x["q"], x["k"], x["v"], x["sinks"], cfg.W, cfg.scale, out, lse)
+            g = torch.Generator(device=dev).manual_seed(1)
+            dout = torch.randn(x["q"].shape, device=dev, generator=g).to(torch.bfloat16)
+            dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+            dsink = torch.empty(cfg.Hq, dtype=torch.float32, device=dev)
+            for _ in range(a.launches):
+                abi.attn_sink_bwd(x["q"], x["k"], x["v"], out, lse, dout, x["sinks"], cfg.W, cfg.scale,
+                                  dq, dk, dv, dsink)
     else:
         if not isinstance(cfg, inputs.Decode):
             raise SystemExit("decode needs a decode workload")
