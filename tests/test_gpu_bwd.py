@@ -70,6 +70,10 @@ CASES = [  # B, L, Hq, Hkv, D, W, sinks
     (1, 517, 6, 2, 128, 1 << 30, "uniform"),
     (2, 129, 4, 1, 128, 33, "none"),
     (1, 190, 4, 2, 128, 100, 20.0),
+    (1, 200, 2, 2, 128, 1, "uniform"),       # W = 1, one query head per kv head
+    (1, 64, 6, 2, 128, 1 << 30, "uniform"),  # three heads per kv head, one query block
+    (1, 1, 4, 2, 128, 5, "uniform"),         # a single position
+    (3, 131, 8, 8, 128, 7, -30.0),           # sinks far below the logits
 ]
 
 
@@ -110,3 +114,24 @@ def test_bwd_prefill_heads_sampled():
     ref = oracle.bwd(inputs.bits(q[:, :, :8]), inputs.bits(k[:, :, :1]), inputs.bits(v[:, :, :1]),
                      s[:8].numpy(), inputs.bits(do[:, :, :8]), W, scale)
     _check([got[0][:, :, :8], got[1][:, :, :1], got[2][:, :, :1], got[3][:8]], ref, "prefill heads")
+
+
+def test_bwd_strided_packed_qkv():
+    """q, k, v as head slices of one packed [B, L, Hq + 2 Hkv, D] projection and
+    dq/dk/dv written into slices of a packed gradient: strides other than the
+    contiguous ones reach the tensor maps and the row loads."""
+    B, L, Hq, Hkv, D, W = 2, 150, 4, 2, 128, 40
+    q, k, v, do, s = _case(B, L, Hq, Hkv, D, seed=77)
+    scale = 1.0 / np.sqrt(D)
+    ref = oracle.bwd(inputs.bits(q), inputs.bits(k), inputs.bits(v), s.numpy(), inputs.bits(do), W, scale)
+    qkv = torch.cat([q, k, v], dim=2).to(DEV)
+    qs, ks, vs = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:]
+    o, lse = swl.fwd(qs, ks, vs, s.to(DEV), W, scale)
+    g = torch.full((B, L, Hq + 2 * Hkv, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    dq, dk, dv = g[:, :, :Hq], g[:, :, Hq:Hq + Hkv], g[:, :, Hq + Hkv:]
+    dsink = torch.empty(Hq, device=DEV)
+    swl.attn_sink_bwd(qs, ks, vs, o, lse, do.to(DEV), s.to(DEV), W, scale, dq, dk, dv, dsink)
+    torch.cuda.synchronize()
+    assert swl.attn_sink_get_status() == 0
+    got = [t.float().cpu().numpy() for t in (dq, dk, dv, dsink)]
+    _check(got, ref, "strided bwd")
