@@ -396,8 +396,8 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   uint64_t *s_full = q_empty + 2;           // [NH][2] S^w ready in S buffer
   uint64_t *p_full = s_full + 2 * NH;       // [NH][2] P^w ready in S buffer (O^w rescaled)
   uint64_t *pv_done = p_full + 2 * NH;      // [NH] one PV^w finished
-  uint64_t *o_full = pv_done + NH;          // every MMA of a unit finished
-  uint64_t *o_drained = o_full + 1;         // [NH] O^w of a unit read out of TMEM
+  uint64_t *o_full = pv_done + NH;          // [NH] a unit's last PV^w finished
+  uint64_t *o_drained = o_full + NH;        // [NH] O^w of a unit read out of TMEM
   uint64_t *mma_done = o_drained + NH;      // every MMA of the CTA finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
@@ -457,9 +457,9 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         mbar_init(&p_full[2 * w + buf], 128);
       }
       mbar_init(&pv_done[w], 1);
+      mbar_init(&o_full[w], 1);
       mbar_init(&o_drained[w], 128);
     }
-    mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -579,55 +579,64 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         tc_fence_after();
         return ok;
       };
+      // S^w_g = Q^w K^T into S buffer g%kSBuf of head w, Q from buffer qbuf
+      // (overwriting the P^w that the PV^w issued before it has consumed: the
+      // tensor pipe runs in order)
+      auto issue_s = [&](int w, int ks, int g, int qbuf) {
+        const uint32_t a0 = q_lo + ((qbuf * C::kQBufBytes + w * C::kQTileBytes) >> 4);
+        const uint32_t b0 = ring_lo_k + ks * (C::kTileBytes >> 4);
+        const uint32_t d = tmem + C::kSCol(w, g % C::kSBuf);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
+          umma_ss_w(d, a0 + (kk >> 2) * (kBM * 128 >> 4) + (kk & 3) * 2, desc_hi,
+                    b0 + (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2, desc_hi, idesc_qk,
+                    kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[2 * w + g % C::kSBuf]);
+      };
+      // O^w += P^w_g V with P^w_g (bf16 pairs) in the first BN/2 columns of
+      // its S buffer; j = 0 starts a unit's O^w
+      auto issue_pv = [&](int w, int vs, int g, int j) {
+        const uint32_t b0 = ring_lo_v + vs * (C::kTileBytes >> 4);
+        const uint32_t a0 = tmem + C::kSCol(w, g % C::kSBuf);
+        const uint32_t d = tmem + C::kOCol(w);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts_w(d, a0 + kk * 8, b0 + kk * (16 * 128 >> 4), desc_hi, idesc_pv,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&pv_done[w]);
+      };
       int jg = 0;                            // tiles of earlier units (barrier phases)
+      bool pre = false;                      // this unit's first S (every head) already issued
       for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const Unit t = unit_at(u);
         if (packed && t.n_tiles <= 0) continue;   // ul counts the units that are not empty
         const int qb = ul & 1;
-        if (!mbar_wait(&q_full[qb], static_cast<uint32_t>(ul >> 1) & 1u, ctx, kWhereQ)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // S^w_j = Q^w K_j^T into S buffer (jg+j)%kSBuf of head w (overwriting
-        // the P^w that the PV^w issued before it has consumed: the tensor pipe
-        // runs in order)
-        auto issue_s = [&](int w, int ks, int j) {
-          const int g = jg + j;
-          const uint32_t a0 = q_lo + ((qb * C::kQBufBytes + w * C::kQTileBytes) >> 4);
-          const uint32_t b0 = ring_lo_k + ks * (C::kTileBytes >> 4);
-          const uint32_t d = tmem + C::kSCol(w, g % C::kSBuf);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
-            umma_ss_w(d, a0 + (kk >> 2) * (kBM * 128 >> 4) + (kk & 3) * 2, desc_hi,
-                      b0 + (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2, desc_hi, idesc_qk,
-                      kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[2 * w + g % C::kSBuf]);
-        };
-        // O^w += P^w_j V_j with P^w_j (bf16 pairs) in the first BN/2 columns
-        // of its S buffer
-        auto issue_pv = [&](int w, int vs, int j) {
-          const int g = jg + j;
-          const uint32_t b0 = ring_lo_v + vs * (C::kTileBytes >> 4);
-          const uint32_t a0 = tmem + C::kSCol(w, g % C::kSBuf);
-          const uint32_t d = tmem + C::kOCol(w);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ts_w(d, a0 + kk * 8, b0 + kk * (16 * 128 >> 4), desc_hi, idesc_pv,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&pv_done[w]);
-        };
+        // With one S buffer per head, the next unit's first S^w is issued
+        // right behind this unit's last PV^w, so that it is ready when the
+        // warpgroup finishes this unit's epilogue.
+        int un = u + static_cast<int>(gridDim.x);
+        if constexpr (packed)
+          while (un < p.num_units && unit_at(un).n_tiles <= 0) un += gridDim.x;
+        const bool early_next = C::kSBuf == 1 && un < p.num_units;
         int ks = 0, vs = 0;
-        for (int jj = 0; ok && jj < C::kSBuf && jj < t.n_tiles; ++jj) {
-          if (!acquire(ks)) break;
-          for (int w = 0; w < NH; ++w) issue_s(w, ks, jj);
-          umma_commit(&empty[ks]);
+        if (!pre) {
+          if (!mbar_wait(&q_full[qb], static_cast<uint32_t>(ul >> 1) & 1u, ctx, kWhereQ)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int jj = 0; ok && jj < C::kSBuf && jj < t.n_tiles; ++jj) {
+            if (!acquire(ks)) break;
+            for (int w = 0; w < NH; ++w) issue_s(w, ks, jg + jj, qb);
+            umma_commit(&empty[ks]);
+          }
         }
         for (int j = 0; ok && j < t.n_tiles; ++j) {
           const int g = jg + j;
           const bool more = j + C::kSBuf < t.n_tiles;
+          const bool last = j == t.n_tiles - 1;
           if (!acquire(vs)) break;
           for (int w = 0; w < NH; ++w) {
             if (!mbar_wait(&p_full[2 * w + g % C::kSBuf], static_cast<uint32_t>(g / C::kSBuf) & 1u,
@@ -643,17 +652,29 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
               break;
             }
             tc_fence_after();
-            issue_pv(w, vs, j);
+            issue_pv(w, vs, g, j);
+            if (last) umma_commit(&o_full[w]);   // this unit's O^w is complete
             if (w == NH - 1) umma_commit(&empty[vs]);
-            if (more) {
-              if (w == 0 && !acquire(ks)) break;
-              issue_s(w, ks, j + C::kSBuf);
+            // the S that this PV frees the buffer for: this unit's S_{j+kSBuf},
+            // or (one buffer, last tile) the next unit's S_0, global tile g + 1
+            if (more || (last && early_next)) {
+              if (w == 0) {
+                if (!more) {
+                  if (!mbar_wait(&q_full[qb ^ 1], static_cast<uint32_t>((ul + 1) >> 1) & 1u, ctx, kWhereQ)) {
+                    ok = false;
+                    break;
+                  }
+                  tc_fence_after();
+                }
+                if (!acquire(ks)) break;
+              }
+              issue_s(w, ks, g + C::kSBuf, more ? qb : qb ^ 1);
               if (w == NH - 1) umma_commit(&empty[ks]);
             }
           }
         }
+        pre = early_next;
         jg += t.n_tiles;
-        umma_commit(o_full);                 // this unit's O is complete
         ++ul;
       }
       // Every tensor-core operation of this CTA has finished before teardown.
@@ -734,7 +755,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         }
       }
       jg += t.n_tiles;
-      if (ok) ok = warp_wait(o_full, static_cast<uint32_t>(ul) & 1u, ctx, kWhereO);
+      if (ok) ok = warp_wait(&o_full[w], static_cast<uint32_t>(ul) & 1u, ctx, kWhereO);
       if (!ok) break;
       tc_fence_after();
       // ---- sink epilogue (page "cf-1.com/news/6055759", fix 2) ----
@@ -755,11 +776,8 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       // the next unit's PV^w may overwrite it.
       uint8_t *stage = sQ + qb * C::kQBufBytes + w * C::kQTileBytes;
       const bool direct = packed && t.m0 + kBM > t.len;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(lane_base + o_col + c * 32, o);
-        tmem_wait_ld();
+      // the next 32-column chunk is read while this one is converted
+      auto convert = [&](int c, const uint32_t (&o)[32]) {
         uint8_t *chunk = stage + (c >> 1) * (kBM * 128) + r * 128;
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
@@ -776,6 +794,30 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
             const int unit = (c & 1) * 4 + uu;      // 16-byte unit within the 128-byte row
             *reinterpret_cast<uint4 *>(chunk + ((unit ^ (r & 7)) << 4)) = v;
           }
+        }
+      };
+      static_assert(D % 64 == 0, "chunks are converted in pairs");
+      if constexpr (packed) {
+        // (the packed kernel keeps one chunk in flight: its row-by-row stores
+        // leave no registers for a second)
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + o_col + c * 32, o);
+          tmem_wait_ld_dep(o);
+          convert(c, o);
+        }
+      } else {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(lane_base + o_col, oa);
+#pragma unroll
+        for (int c = 0; c < D / 32; c += 2) {
+          tmem_wait_ld_dep(oa);
+          tmem_ld32(lane_base + o_col + (c + 1) * 32, ob);
+          convert(c, oa);
+          tmem_wait_ld_dep(ob);
+          if (c + 2 < D / 32) tmem_ld32(lane_base + o_col + (c + 2) * 32, oa);
+          convert(c + 1, ob);
         }
       }
       tc_fence_before();
