@@ -139,6 +139,24 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- our arm
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank timings over all ranks (every rank
+    calls it, in the same order); a no-op for one rank."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_rate(work_per_rank, world, seconds):
+    """Whole-job rate: every rank does the same work (weak scaling), timed as
+    the slowest rank's time."""
+    return world * work_per_rank / seconds
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -360,23 +378,20 @@ def run_ours(args, rank, world, local_rank):
     del bdo, bdq, bdk, bdv
 
     # ---- max over ranks ----
-    times = torch.tensor([t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8, t_bwd], dtype=torch.float64,
-                         device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8, t_bwd = times.tolist()
+    t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8, t_bwd = max_over_ranks(
+        [t_fwd, t_dec, t_all, t_e2e, t_paged, t_varlen, t_fp8, t_bwd], world, dev)
 
     if rank != 0:
         return
     peaks, peak_src = load_peaks()
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    fwd_tflops = world * K * fwd_flops / t_fwd / 1e12
+    fwd_tflops = aggregate_rate(K * fwd_flops, world, t_fwd) / 1e12
     per_launch_fwd = t_fwd / K
     per_launch_dec = t_dec / K
     achieved_fwd = fwd_flops / per_launch_fwd / 1e12
     achieved_dec = dbytes / per_launch_dec / 1e9
-    dec_gbs = world * K * dbytes / t_dec / 1e9
+    dec_gbs = aggregate_rate(K * dbytes, world, t_dec) / 1e9
     line = {
         "metric": METRIC,
         "value": round(fwd_tflops, 3),
@@ -408,22 +423,22 @@ def run_ours(args, rank, world, local_rank):
                                 "traffic": profiled_traffic("decode_split", [
                                     "sliding_window_learned_b200/csrc/decode.cu",
                                     "sliding_window_learned_b200/csrc/ptx.cuh"])}},
-        "decode_paged": {"value": round(world * Kp * dbytes / t_paged / 1e9, 2), "unit": "GB/s",
+        "decode_paged": {"value": round(aggregate_rate(Kp * dbytes, world, t_paged) / 1e9, 2), "unit": "GB/s",
                          "page": page, "ms_per_call": round(t_paged / Kp * 1e3, 4),
                          "frac": round(dbytes / (t_paged / Kp) / 1e9 / hbm_peak, 4),
                          "what": "attn_sink_decode_paged on the decode workload, cache in 256-position "
                                  "pages at random pool positions"},
-        "decode_fp8": {"value": round(world * Kp * dbytes8 / t_fp8 / 1e9, 2), "unit": "GB/s",
+        "decode_fp8": {"value": round(aggregate_rate(Kp * dbytes8, world, t_fp8) / 1e9, 2), "unit": "GB/s",
                        "ms_per_call": round(t_fp8 / Kp * 1e3, 4),
                        "frac": round(dbytes8 / (t_fp8 / Kp) / 1e9 / hbm_peak, 4),
                        "what": "attn_sink_decode_fp8 on the decode workload, cache quantised to e4m3 per "
                                "kv head (bytes counted at one per element)"},
-        "fwd_varlen": {"value": round(world * Kv * vl_flops / t_varlen / 1e12, 3), "unit": "TFLOP/s",
+        "fwd_varlen": {"value": round(aggregate_rate(Kv * vl_flops, world, t_varlen) / 1e12, 3), "unit": "TFLOP/s",
                        "ms_per_call": round(t_varlen / Kv * 1e3, 5),
                        "frac": round(vl_flops / (t_varlen / Kv) / 1e12 / bf16_peak, 4),
                        "what": "attn_sink_fwd_varlen on 24 packed sequences of U[1, 4096] tokens "
                                f"(T = {vl_T}), Hq32 Hkv4 D128 W513, L2 flushed before each call"},
-        "bwd": {"value": round(world * Kb * 2.5 * fwd_flops / t_bwd / 1e12, 3), "unit": "TFLOP/s",
+        "bwd": {"value": round(aggregate_rate(Kb * 2.5 * fwd_flops, world, t_bwd) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_call": round(t_bwd / Kb * 1e3, 5),
                 "frac": round(2.5 * fwd_flops / (t_bwd / Kb) / 1e12 / bf16_peak, 4),
                 "traffic_main_pass": profiled_traffic("bwd_tc", ["sliding_window_learned_b200/csrc/bwd_tc.cu",
@@ -432,7 +447,7 @@ def run_ours(args, rank, world, local_rank):
                 "what": "attn_sink_bwd (dq, dk, dv, dsink) on the prefill workload, O and LSE from "
                         "attn_sink_fwd; useful FLOPs = 10 D per visible pair (2.5x the forward's), "
                         "L2 flushed before each call"},
-        "e2e": {"value": round(world * Ke * fwd_flops / t_e2e / 1e12, 4), "unit": "TFLOP/s",
+        "e2e": {"value": round(aggregate_rate(Ke * fwd_flops, world, t_e2e) / 1e12, 4), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "attn_sink_fwd with pinned host inputs copied in and O, LSE copied out each step"},
         "gpu_launches": K * 4,
