@@ -359,7 +359,10 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       // zeros.  Then the FP8 stage goes back to the producer at once.
       const uint8_t *src = smem + s * C::kStageBytes;
       uint8_t *conv = smem + C::kConvOffset;
-      const int row = key_w + (lane >> 1);
+      // lanes l and l + 16 share a row (one half each), so that the eight
+      // lanes of each 16-byte store phase cover eight rows: eight distinct
+      // swizzled slots, no bank conflict
+      const int row = key_w + (lane & 15);
       const bool valid = row >= si.nskip && row < si.nvalid;
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
@@ -367,7 +370,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
         for (int c8 = 0; c8 < C::kChunks8; ++c8) {
 #pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
-            const int u = (lane & 1) * 4 + uu;     // 16-byte unit (16 elements) of the 128-byte row
+            const int u = (lane >> 4) * 4 + uu;    // 16-byte unit (16 elements) of the 128-byte row
             uint4 x = make_uint4(0, 0, 0, 0);
             if (valid)
               x = *reinterpret_cast<const uint4 *>(src + kv * C::kTileBytes + c8 * C::kTK * 128 + row * 128 +

@@ -5,7 +5,8 @@ captures (Nsight Compute) of a single kernel on a bounded device footprint.
   python -m sliding_window_learned_b200.ncu_driver --op decode --workload decode-small --launches 3
   python -m sliding_window_learned_b200.ncu_driver --op bwd --workload prefill --launches 2
 
-(--op bwd runs one forward for O and LSE, then the backward passes.)
+(--op bwd runs one forward for O and LSE, then the backward passes; --op
+decode_fp8 quantises the workload's cache to e4m3 per kv head first.)
 
 It prints no timings (numbers taken under a profiler are not measurements);
 it exits non-zero if the device reports an error.
@@ -33,7 +34,7 @@ WORKLOADS = {
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["fwd", "decode", "bwd"], required=True)
+    ap.add_argument("--op", choices=["fwd", "decode", "bwd", "decode_fp8"], required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
     ap.add_argument("--launches", type=int, default=3)
     a = ap.parse_args(argv)
@@ -64,9 +65,22 @@ def main(argv=None) -> int:
             raise SystemExit("decode needs a decode workload")
         y = inputs.make_decode(cfg, seed=0, device=dev)
         out = torch.empty_like(y["q"])
-        for _ in range(a.launches):
-            abi.attn_sink_decode(y["q"], y["kcache"], y["vcache"], y["seqlens"], y["sinks"],
-                                 cfg.W, cfg.scale, out)
+        if a.op == "decode_fp8":
+            kd = torch.empty(cfg.Hkv, device=dev)
+            vd = torch.empty(cfg.Hkv, device=dev)
+            k8 = torch.empty(y["kcache"].shape, dtype=torch.float8_e4m3fn, device=dev)
+            v8 = torch.empty_like(k8)
+            for hk in range(cfg.Hkv):
+                for src, dst, d in ((y["kcache"], k8, kd), (y["vcache"], v8, vd)):
+                    xs = src[:, :, hk].float()
+                    d[hk] = torch.nan_to_num(xs, nan=0.0).abs().amax() / 448.0
+                    dst[:, :, hk] = (xs / d[hk]).to(torch.float8_e4m3fn)
+            for _ in range(a.launches):
+                abi.attn_sink_decode_fp8(y["q"], k8, v8, kd, vd, y["seqlens"], y["sinks"], cfg.W, cfg.scale, out)
+        else:
+            for _ in range(a.launches):
+                abi.attn_sink_decode(y["q"], y["kcache"], y["vcache"], y["seqlens"], y["sinks"],
+                                     cfg.W, cfg.scale, out)
     torch.cuda.synchronize()
     rc = abi.attn_sink_get_status()
     print("ok" if rc == 0 else f"device status {rc}")
