@@ -154,12 +154,12 @@ struct StageInfo {
 // converted to f16 after a power-of-two scale that puts its largest magnitude
 // in [2^13, 2^14) (undone in the softmax scale), and P is f16.
 // An FP8 cache delivers a key in half the bytes, so at D = 128 its tiles are
-// 128 keys for 8 consumer warps (two per SM sub-partition), which keeps the
-// consumers ahead of HBM; the merge buffer then lives in the conversion tile
+// 192 keys for 12 consumer warps (three per SM sub-partition, to hide the
+// conversion's latency); the merge buffer then lives in the conversion tile
 // (free at an item's end).
 template <int D, int NT, bool kF8>
 struct DCfg {
-  static constexpr int kCW = (kF8 && D == 128) ? 8 : kConsumerWarps;   // consumer warps
+  static constexpr int kCW = (kF8 && D == 128) ? 12 : kConsumerWarps;  // consumer warps
   static constexpr int kTK = 16 * kCW;                    // keys per tile
   static constexpr int kThreads = (kCW + 1) * 32;         // + the producer warp
   static constexpr bool kMergeInConv = kF8;
@@ -170,7 +170,7 @@ struct DCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
   static constexpr int kConvBytes = kF8 ? 2 * kBf16TileBytes : 0;
   static constexpr int kMergeBytes = kCW * NT * 8 * D * 4;
-  static constexpr int kRingBudget = 196608 - kConvBytes - (kMergeInConv ? 0 : kMergeBytes);
+  static constexpr int kRingBudget = (kF8 ? 221184 : 196608) - kConvBytes - (kMergeInConv ? 0 : kMergeBytes);
   static constexpr int kStages = (kRingBudget / kStageBytes) > 12 ? 12 : (kRingBudget / kStageBytes);
   static constexpr int kConvOffset = kStages * kStageBytes;
   static constexpr int kMergeOffset = kMergeInConv ? kConvOffset : kConvOffset + kConvBytes;
