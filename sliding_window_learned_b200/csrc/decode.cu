@@ -155,11 +155,12 @@ struct StageInfo {
 // in [2^13, 2^14) (undone in the softmax scale), and P is f16.
 // An FP8 cache delivers a key in half the bytes, so at D = 128 its tiles are
 // 192 keys for 12 consumer warps (three per SM sub-partition, to hide the
-// conversion's latency); the merge buffer then lives in the conversion tile
-// (free at an item's end).
+// conversion's latency; 128 keys and 8 warps for groups of more than 8 heads,
+// whose accumulators need the registers); the merge buffer then lives in the
+// conversion tile (free at an item's end).
 template <int D, int NT, bool kF8>
 struct DCfg {
-  static constexpr int kCW = (kF8 && D == 128) ? 12 : kConsumerWarps;  // consumer warps
+  static constexpr int kCW = (kF8 && D == 128) ? (NT == 1 ? 12 : 8) : kConsumerWarps;   // consumer warps
   static constexpr int kTK = 16 * kCW;                    // keys per tile
   static constexpr int kThreads = (kCW + 1) * 32;         // + the producer warp
   static constexpr bool kMergeInConv = kF8;
@@ -236,8 +237,11 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
   __syncthreads();
 
   if (warp == C::kCW) {
+    const bool small_pages = !kF8 && p.page != 0 && p.page < C::kTK;
     // -------------------------------------------------------------- producer
-    if (lane == 0) {
+    // Contiguous cache, FP8 cache, or pages of at least a tile: one lane
+    // issues everything.
+    if (!small_pages && lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const int total_items = p.ctrl[0] * p.Hkv;
@@ -326,6 +330,111 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       if (ok) {
         const int s = acquire();
         if (ok) {
+          info[s].flags = 4;
+          mbar_arrive(&full[s]);
+        }
+      }
+    }
+    // Pages smaller than a tile (several boxes per tile): the whole warp
+    // follows one control flow; lane 0 claims work, waits for free stages and
+    // arms their barriers (results shared by shuffle), and the copies of a
+    // tile (one per page box, chunk and K/V) are issued by one lane each.
+    if (small_pages) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
+      const int total_items = p.ctrl[0] * p.Hkv;
+      int slot = 0;
+      bool ok = true;
+      auto acquire = [&]() -> int {
+        const int s = slot % C::kStages;
+        const uint32_t use = static_cast<uint32_t>(slot / C::kStages);
+        bool good = true;
+        if (lane == 0 && slot >= C::kStages && !mbar_wait(&empty[s], (use & 1u) ^ 1u, ctx, kWhereEmpty))
+          good = false;
+        ok = ok && __shfl_sync(0xffffffffu, good, 0);
+        ++slot;
+        return s;
+      };
+      while (ok) {
+        int w = 0;
+        if (lane == 0) w = atomicAdd(p.work_counter, 1);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (w >= total_items) break;
+        const int g = w / p.Hkv, hk = w - g * p.Hkv;
+        int lo = 0, hi = p.B - 1;  // last b with base[b] <= g
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (p.base[mid] <= g) lo = mid; else hi = mid - 1;
+        }
+        const int b = lo;
+        const int split = g - p.base[b];
+        const int n = min(max(p.seqlens[b], 0), p.Smax);
+        const int vis0 = max(0, n - p.W);
+        const int ks = vis0 / p.align * p.align + split * p.chunk;
+        const int ke = min(n, ks + p.chunk);
+        const int nt = (ke - ks + C::kTK - 1) / C::kTK;
+        const int nbox = p.page == 0 ? 1 : C::kTK / min(C::kTK, p.page);   // boxes per tile (paged)
+        for (int t = 0; ok && t < nt; ++t) {
+          const int key0 = ks + t * C::kTK;
+          // Paged cache: lane r < nbox reads box r's page number before the
+          // stage wait, so that the table reads overlap it.
+          int blk = 0;
+          if (p.page != 0 && lane < nbox) {
+            const int lp = (key0 + lane * (C::kTK / nbox)) >> p.page_shift;
+            blk = lp < p.max_pages ? p.block_table[static_cast<int64_t>(b) * p.bt_s0 + lp] : -1;
+          }
+          const int s = acquire();
+          if (!ok) break;
+          uint8_t *dst = smem + s * C::kStageBytes;
+          if (lane == 0) {
+            StageInfo &si = info[s];
+            si.b = b;
+            si.hk = hk;
+            si.split = split;
+            si.key0 = key0;
+            si.nvalid = min(C::kTK, ke - key0);
+            si.nskip = max(0, vis0 - key0);
+            si.flags = (t == 0 ? 1 : 0) | (t == nt - 1 ? 2 : 0);
+            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          }
+          __syncwarp();
+          if (kF8) {
+            if (lane == 0)
+              for (int c = 0; c < C::kChunks8; ++c) {
+                tma_load_4d(dst + c * C::kTK * 128, &tmK, &full[s], c * 128, hk, key0, b);
+                tma_load_4d(dst + C::kTileBytes + c * C::kTK * 128, &tmV, &full[s], c * 128, hk, key0, b);
+              }
+          } else if (p.page == 0) {
+            if (lane == 0)
+              for (int c = 0; c < C::kChunks; ++c) {
+                tma_load_4d(dst + c * C::kTK * 128, &tmK, &full[s], c * 64, hk, key0, b);
+                tma_load_4d(dst + C::kTileBytes + c * C::kTK * 128, &tmV, &full[s], c * 64, hk, key0, b);
+              }
+          } else {
+            // key0 is a multiple of 64 here, so each box of min(64, page) rows
+            // lies in one page.  A table entry outside the pool (or a page
+            // number past the table, for rows beyond the sequence end) loads
+            // zero rows: the box is out of range and filled, and it still
+            // delivers its bytes.  Lane (r, c, kv) issues box r's chunk c of
+            // K (kv = 0) or V (kv = 1).
+            const int rows = C::kTK / nbox;
+            const int copies = nbox * C::kChunks * 2;
+            const int r = lane / (C::kChunks * 2), c = (lane >> 1) % C::kChunks, kv = lane & 1;
+            const int blk_r = __shfl_sync(0xffffffffu, blk, r < nbox ? r : 0);
+            if (lane < copies) {
+              const int r0 = r * rows;
+              const int row_in_page = (key0 + r0) & (p.page - 1);
+              tma_load_4d(dst + kv * C::kTileBytes + c * C::kTK * 128 + r0 * 128, kv ? &tmV : &tmK, &full[s],
+                          c * 64, hk, row_in_page, blk_r);
+            }
+          }
+        }
+      }
+      if (ok) {
+        const int s = acquire();
+        if (ok && lane == 0) {
           info[s].flags = 4;
           mbar_arrive(&full[s]);
         }
