@@ -456,6 +456,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+        line["decode"]["cpu_baseline"] = cpu_baseline_decode(y, dcfg)
+        line["bwd"]["cpu_baseline"] = cpu_baseline_bwd(x, pcfg)
     print(json.dumps(line), flush=True)
 
 
@@ -502,6 +504,49 @@ def cpu_baseline(budget_s: float = 10.0):
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"{n_rows} random (b, i, h) rows of {inputs.PREFILL.name}, fp64, {dt:.1f} s"}
+
+
+def cpu_baseline_decode(y, cfg, n_seq=2):
+    """The oracle's decode, as it stands, on a bounded sample of the decode
+    workload (n_seq of its sequences, every head); GB/s of their algorithmic
+    bytes."""
+    import oracle
+    oracle.build()
+    sl = y["seqlens"].cpu().numpy()
+    pick = np.sort(np.random.default_rng(7).choice(cfg.B, size=n_seq, replace=False))
+    nmax = int(sl[pick].max())
+    q = inputs.bits(y["q"][pick].cpu())
+    kb = inputs.bits(y["kcache"][pick, :nmax].cpu())
+    vb = inputs.bits(y["vcache"][pick, :nmax].cpu())
+    nbytes = float(sl[pick].sum()) * cfg.Hkv * cfg.D * 2 * 2 + 2 * n_seq * cfg.Hq * cfg.D * 2
+    t0 = time.perf_counter()
+    oracle.decode(q, kb, vb, sl[pick].astype(np.int32), y["sinks"].cpu().numpy(), cfg.W, cfg.scale)
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_seq} sequences (n = {', '.join(str(int(n)) for n in sl[pick])}) of {cfg.name}, "
+                      f"every head, fp64, {dt:.1f} s"}
+
+
+def cpu_baseline_bwd(x, cfg, L=2048):
+    """The oracle's backward, as it stands, on a bounded slice of the prefill
+    workload: the first L positions of batch 0 and the query heads of kv head
+    0; useful TFLOP/s of the slice (2.5x its forward FLOPs)."""
+    import torch
+
+    import oracle
+    G = cfg.Hq // cfg.Hkv
+    q, k, v = (x["q"][:1, :L, :G].cpu(), x["k"][:1, :L, :1].cpu(), x["v"][:1, :L, :1].cpu())
+    g = torch.Generator().manual_seed(3)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    flops = 2.5 * 4.0 * cfg.D * G * float(np.minimum(np.arange(L) + 1, cfg.W).sum())
+    t0 = time.perf_counter()
+    oracle.bwd(inputs.bits(q), inputs.bits(k), inputs.bits(v), x["sinks"][:G].cpu().numpy(), inputs.bits(do),
+               cfg.W, cfg.scale)
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"positions 0..{L - 1} of batch 0, query heads 0..{G - 1} (kv head 0) of {cfg.name}, "
+                      f"fp64 autograd, {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
