@@ -797,9 +797,10 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         }
       };
       static_assert(D % 64 == 0, "chunks are converted in pairs");
-      if constexpr (packed) {
+      if constexpr (packed || NH == 1) {
         // (the packed kernel keeps one chunk in flight: its row-by-row stores
-        // leave no registers for a second)
+        // leave no registers for a second; so does the one-head kernel, which
+        // has no register reallocation and measured 1.6 % slower with two)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
