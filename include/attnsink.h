@@ -164,13 +164,13 @@ int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k,
  *   dk, dv      [B, L, Hkv, D] bf16, written completely (summed over the
  *               query heads of each kv head)
  *   dsink       [Hq] f32, summed over the batch
- * D in {64, 128}.  Workspace, from the library's stream-ordered pool: an
- * fp32 dq accumulator and the row sums, B*L*Hq*(D+1)*4 bytes, and at D = 128
- * fp32 dk and dv accumulators, 2*B*L*Hkv*D*4 bytes more.  D = 128 runs on the
- * 5th-generation tensor cores (tcgen05, TMEM accumulators); D = 64 on
- * warp-level (mma.sync) products.  Both accumulate in fp32 and round P and dS
- * to bf16 for the products.  Launches: a row kernel, the main pass, then the
- * fp32 -> bf16 conversions; no host synchronisation.
+ * D in {64, 128}.  Workspace, from the library's stream-ordered pool: fp32
+ * dq accumulator and row sums, B*L*Hq*(D+1)*4 bytes, and fp32 dk and dv
+ * accumulators, 2*B*L*Hkv*D*4 bytes.  The main pass runs on the
+ * 5th-generation tensor cores (tcgen05, TMEM accumulators), accumulating in
+ * fp32 with P and dS rounded to bf16 for the products.  Launches: a row
+ * kernel, the main pass, then the fp32 -> bf16 conversions; no host
+ * synchronisation.
  */
 int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
                   const attn_tensor *o, const attn_tensor *lse, const attn_tensor *dout,

@@ -1,6 +1,6 @@
 // bwd_tc.cu -- backward pass of sliding-window attention with a learned
 // per-head sink on the 5th-generation tensor cores (tcgen05, TMEM, TMA), head
-// dimension 128.  The gradients are those of bwd.cu (page "Dao-AILab/
+// dimension 64 or 128.  The gradients are those of bwd.cu (page "Dao-AILab/
 // flash-attention" contributor guide: the FA4 backward kernels and issue
 // #2969):
 //   P_ij = exp(s_ij - LSE_i), Dsum_i = dO_i . O_i,
@@ -14,9 +14,10 @@
 // with fp32 accumulators in TMEM:
 //   S^T  = K Q^T      [128 keys x 64 queries]   A = K (smem), B = Q (smem)
 //   dP^T = V dO^T     [128 x 64]                A = V, B = dO
-//   dV  += P^T dO     [128 keys x 128]          A = P^T (bf16, TMEM), B = dO (smem, N-major)
-//   dK  += dS^T Q     [128 x 128]               A = dS^T (bf16, TMEM), B = Q (smem, N-major)
+//   dV  += P^T dO     [128 keys x D]            A = P^T (bf16, TMEM), B = dO (smem, N-major)
+//   dK  += dS^T Q     [128 x D]                 A = dS^T (bf16, TMEM), B = Q (smem, N-major)
 //   dQ^T = K^T dS^T   [128 channels x 64]       A = K (smem, M-major), B = dS^T (smem, N-major)
+//                     (at D = 64 channels 64..127 are padding)
 // All five have M = 128 (keys or channels on the TMEM lanes); dQ is formed
 // transposed so that it needs no 64-row accumulator.  P^T and dS^T live in
 // their own TMEM columns, so the next step's S^T and dP^T are computed while
@@ -49,7 +50,6 @@
 namespace attnsink {
 namespace {
 
-constexpr int kD = 128;
 constexpr int kBK = 128;                        // keys per unit (TMEM lanes)
 constexpr int kBQ = 64;                         // queries per step
 constexpr int kThreads = 512;
@@ -64,29 +64,41 @@ static_assert(128 * (2 * kRegsSoftmax + kRegsDrain + kRegsOther) <= kRegsLaunch 
 constexpr uint32_t kBarTmem = 1, kBarDrain = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDS = 160, kColDV = 192, kColDK = 320,
-                   kColDQ = 448, kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColDP = 64, kColP = 128, kColDS = 160, kTmemCols = 512;
 
 // Pipeline depths: Q/dO ring slots (the producer runs kStages - 1 steps
 // ahead), K/V buffers (2: the next unit's K, V load during this unit).
 constexpr int kStages = 3, kKVBuf = 1;
 
-// shared memory, from a 1024-byte aligned base (128-byte swizzled tiles)
-constexpr int kKVTile = kBK * kD * 2;           // a K or V tile: two 64-channel chunks of 128 rows
-constexpr int kQTile = kBQ * kD * 2;            // a Q or dO tile: two chunks of 64 rows
 constexpr int kDSTile = kBK * kBQ * 2;          // dS^T: 128 key rows of 64 queries
-constexpr int kOffK = 0;                        // [kKVBuf] K tiles (units alternate)
-constexpr int kOffV = kOffK + kKVBuf * kKVTile; // [kKVBuf] V tiles
-constexpr int kOffQ = kOffV + kKVBuf * kKVTile; // [kStages] Q tiles (ring slots)
-constexpr int kOffDO = kOffQ + kStages * kQTile;      // [kStages] dO tiles
-constexpr int kOffDS = kOffDO + kStages * kQTile;     // [2] dS^T tiles (steps alternate)
-constexpr int kOffRow = kOffDS + 2 * kDSTile;   // [kStages][LSE*log2e x 64, Dsum x 64] f32
-constexpr int kOffStage = kOffRow + kStages * 2 * kBQ * 4;   // dQ tile [64 queries][128] f32
-constexpr int kOffBar = kOffStage + kBQ * kD * 4;
-static_assert(kOffStage % 128 == 0, "bulk-copy staging alignment");
 constexpr int kBarBytes = 256;
-constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;   // + alignment slack
-static_assert(kSmemBytes <= 227 * 1024, "shared-memory budget");
+
+// Layout for head dimension D (64 or 128).  TMEM: dV and dK take D columns
+// each after the fixed S^T/dP^T/P^T/dS^T columns, dQ^T 64 columns after them
+// (dQ^T keeps M = 128: at D = 64 its lanes 64..127 are computed from the
+// shared memory after the K tile and never read).  Shared memory, from a
+// 1024-byte aligned base (128-byte swizzled tiles).
+template <int D>
+struct BCfg {
+  static_assert(D == 64 || D == 128, "head dimension");
+  static constexpr uint32_t kColDV = 192, kColDK = kColDV + D, kColDQ = kColDK + D;
+  static_assert(kColDQ + kBQ <= kTmemCols, "TMEM budget");
+  static constexpr int kKVTile = kBK * D * 2;           // a K or V tile: D/64 chunks of 128 rows
+  static constexpr int kQTile = kBQ * D * 2;            // a Q or dO tile: D/64 chunks of 64 rows
+  static constexpr int kOffK = 0;                       // [kKVBuf] K tiles
+  static constexpr int kOffV = kOffK + kKVBuf * kKVTile;      // [kKVBuf] V tiles
+  static constexpr int kOffQ = kOffV + kKVBuf * kKVTile;      // [kStages] Q tiles (ring slots)
+  static constexpr int kOffDO = kOffQ + kStages * kQTile;     // [kStages] dO tiles
+  static constexpr int kOffDS = kOffDO + kStages * kQTile;    // [2] dS^T tiles (steps alternate)
+  static constexpr int kOffRow = kOffDS + 2 * kDSTile;        // [kStages][LSE*log2e x 64, Dsum x 64] f32
+  static constexpr int kOffStage = kOffRow + kStages * 2 * kBQ * 4;   // dQ tile [64 queries][D] f32
+  static constexpr int kOffBar = kOffStage + kBQ * D * 4;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;       // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "shared-memory budget");
+  static_assert(kOffStage % 128 == 0, "bulk-copy staging alignment");
+};
+
+
 
 enum : int { kWhereKv = 201, kWhereFull = 202, kWhereEmpty = 203, kWhereS = 204, kWhereP = 205,
              kWhereDq = 206, kWhereDkv = 207 };
@@ -140,17 +152,19 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmDQ, const Params p) {
+  using C = BCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  uint8_t *sK = smem + kOffK, *sV = smem + kOffV, *sQ = smem + kOffQ, *sDO = smem + kOffDO;
-  uint8_t *sDS = smem + kOffDS;
-  float *sRow = reinterpret_cast<float *>(smem + kOffRow);
-  uint64_t *kv_full = reinterpret_cast<uint64_t *>(smem + kOffBar);   // [kKVBuf] K, V of a unit landed
+  uint8_t *sK = smem + C::kOffK, *sV = smem + C::kOffV, *sQ = smem + C::kOffQ, *sDO = smem + C::kOffDO;
+  uint8_t *sDS = smem + C::kOffDS;
+  float *sRow = reinterpret_cast<float *>(smem + C::kOffRow);
+  uint64_t *kv_full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);   // [kKVBuf] K, V of a unit landed
   uint64_t *kv_empty = kv_full + kKVBuf; // [kKVBuf] a unit's last product read its K, V
   uint64_t *full = kv_empty + kKVBuf;    // [kStages] a step's Q, dO (TMA) and rows (32 lanes) landed
   uint64_t *empty = full + kStages;      // [kStages] a step's dV, dK products read its Q, dO
@@ -230,10 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             !mbar_wait(&kv_empty[kvb], static_cast<uint32_t>(ul / kKVBuf - 1) & 1u, ctx, kWhereKv))
           ok = false;
         if (ok) {
-          mbar_arrive_expect_tx(&kv_full[kvb], 2 * kKVTile);
-          for (int c = 0; c < 2; ++c) {
-            tma_load_4d(sK + kvb * kKVTile + c * kBK * 128, &tmK, &kv_full[kvb], c * 64, t.hk, t.j0, t.b);
-            tma_load_4d(sV + kvb * kKVTile + c * kBK * 128, &tmV, &kv_full[kvb], c * 64, t.hk, t.j0, t.b);
+          mbar_arrive_expect_tx(&kv_full[kvb], 2 * C::kKVTile);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(sK + kvb * C::kKVTile + c * kBK * 128, &tmK, &kv_full[kvb], c * 64, t.hk, t.j0, t.b);
+            tma_load_4d(sV + kvb * C::kKVTile + c * kBK * 128, &tmV, &kv_full[kvb], c * 64, t.hk, t.j0, t.b);
           }
           kv_issued = ul + 1;
         }
@@ -266,10 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           row[kBQ + lane + 32 * e] = dr[e];
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[slot], 2 * kQTile);
-          for (int c = 0; c < 2; ++c) {
-            tma_load_4d(sQ + slot * kQTile + c * kBQ * 128, &tmQ, &full[slot], c * 64, h, i0, t.b);
-            tma_load_4d(sDO + slot * kQTile + c * kBQ * 128, &tmDO, &full[slot], c * 64, h, i0, t.b);
+          mbar_arrive_expect_tx(&full[slot], 2 * C::kQTile);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(sQ + slot * C::kQTile + c * kBQ * 128, &tmQ, &full[slot], c * 64, h, i0, t.b);
+            tma_load_4d(sDO + slot * C::kQTile + c * kBQ * 128, &tmDO, &full[slot], c * 64, h, i0, t.b);
           }
         } else {
           mbar_arrive(&full[slot]);
@@ -290,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(kBK, kBQ, 0, 0);    // K-major A and B
-      constexpr uint32_t idesc_kv = umma_idesc_bf16(kBK, kD, 0, 1);    // A in TMEM, B N-major
-      constexpr uint32_t idesc_dq = umma_idesc_bf16(kD, kBQ, 1, 1);    // A M-major, B N-major
+      constexpr uint32_t idesc_kv = umma_idesc_bf16(kBK, D, 0, 1);    // A in TMEM, B N-major
+      constexpr uint32_t idesc_dq = umma_idesc_bf16(128, kBQ, 1, 1);  // A M-major (M = 128 >= D), B N-major
       // 128-byte swizzle, 8-row groups 1024 bytes apart; the leading offset is
       // the distance between 64-element chunks along M or N for the
       // M/N-major operands (K-major operands ignore it)
@@ -322,11 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t acc0 = r.first ? 0u : 1u;
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk)
-          umma_ts_w(tmem + kColDV, tmem + kColP + kk * 8, don_lo + ((r.slot * kQTile + kk * 16 * 128) >> 4), hi,
+          umma_ts_w(tmem + C::kColDV, tmem + kColP + kk * 8, don_lo + ((r.slot * C::kQTile + kk * 16 * 128) >> 4), hi,
                     idesc_kv, kk > 0 ? 1u : acc0);
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk)
-          umma_ts_w(tmem + kColDK, tmem + kColDS + kk * 8, qn_lo + ((r.slot * kQTile + kk * 16 * 128) >> 4), hi,
+          umma_ts_w(tmem + C::kColDK, tmem + kColDS + kk * 8, qn_lo + ((r.slot * C::kQTile + kk * 16 * 128) >> 4), hi,
                     idesc_kv, kk > 0 ? 1u : acc0);
         umma_commit(pbuf_free);
         umma_commit(&empty[r.slot]);
@@ -336,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
-          umma_ss_w(tmem + kColDQ, km_lo + ((r.kvb * kKVTile + kk * 16 * 128) >> 4), hi,
+          umma_ss_w(tmem + C::kColDQ, km_lo + ((r.kvb * C::kKVTile + kk * 16 * 128) >> 4), hi,
                     ds_lo + (((r.g & 1) * kDSTile + kk * 16 * 128) >> 4), hi, idesc_dq, kk > 0 ? 1u : 0u);
         umma_commit(dq_full);
         umma_commit(&dsm_free[r.g & 1]);
@@ -374,16 +388,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
+          for (int kk = 0; kk < D / 16; ++kk) {
             // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
-            const uint32_t ka = ((kvb * kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
-            const uint32_t qa = ((slot * kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
+            const uint32_t ka = ((kvb * C::kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
+            const uint32_t qa = ((slot * C::kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
             umma_ss_w(tmem + kColS, k_lo + ka, hi, q_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t ka = ((kvb * kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
-            const uint32_t qa = ((slot * kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ka = ((kvb * C::kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
+            const uint32_t qa = ((slot * C::kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
             umma_ss_w(tmem + kColDP, v_lo + ka, hi, do_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
           }
           umma_commit(s_full);
@@ -496,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------- dQ^T out of TMEM; dK, dV at the end of a unit
     const int rr = (warp & 3) * 32 + lane;            // TMEM lane: channel (dQ^T), key row (dK, dV)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    float *stage = reinterpret_cast<float *>(smem + kOffStage);
+    float *stage = reinterpret_cast<float *>(smem + C::kOffStage);
     bool ok = true;
     int g = 0, ul = 0;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
@@ -511,8 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         uint32_t x0[32], x1[32];
-        tmem_ld32(lane_base + kColDQ, x0);
-        tmem_ld32(lane_base + kColDQ + 32, x1);
+        tmem_ld32(lane_base + C::kColDQ, x0);
+        tmem_ld32(lane_base + C::kColDQ + 32, x1);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(dq_empty);                        // the next dQ^T may overwrite it
@@ -521,10 +535,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(kBarDrain, 128);
         // dQ^T column -> dQ row-major tile: for each query the warp writes 32
         // consecutive channels
+        if (rr < D) {                                 // (lanes past D hold padding)
 #pragma unroll
-        for (int c = 0; c < 32; ++c) stage[c * kD + rr] = __uint_as_float(x0[c]) * p.scale;
+          for (int c = 0; c < 32; ++c) stage[c * D + rr] = __uint_as_float(x0[c]) * p.scale;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) stage[(32 + c) * kD + rr] = __uint_as_float(x1[c]) * p.scale;
+          for (int c = 0; c < 32; ++c) stage[(32 + c) * D + rr] = __uint_as_float(x1[c]) * p.scale;
+        }
         fence_proxy_async_smem();
         named_barrier_sync(kBarDrain, 128);
         if (rr == 0) {
@@ -539,12 +555,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const int j = t.j0 + rr;
-          const int64_t kv_row = ((static_cast<int64_t>(t.b) * p.L + j) * p.Hkv + t.hk) * kD;
+          const int64_t kv_row = ((static_cast<int64_t>(t.b) * p.L + j) * p.Hkv + t.hk) * D;
 #pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t k32[32], v32[32];
-            tmem_ld32(lane_base + kColDK + c * 32, k32);
-            tmem_ld32(lane_base + kColDV + c * 32, v32);
+            tmem_ld32(lane_base + C::kColDK + c * 32, k32);
+            tmem_ld32(lane_base + C::kColDV + c * 32, v32);
             tmem_wait_ld();
             if (j < p.L) {
 #pragma unroll
@@ -575,19 +591,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-}  // namespace
-
-cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float *dk_acc, float *dv_acc,
-                               cudaStream_t stream) {
-  if (a.D != kD) return cudaErrorInvalidValue;
+template <int D>
+cudaError_t launch_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float *dk_acc, float *dv_acc,
+                      cudaStream_t stream) {
+  using C = BCfg<D>;
   alignas(64) CUtensorMap mq, mk, mv, mdo, mdq;
   cudaError_t e;
-  if ((e = make_tma_bshd(&mq, a.q, a.B, a.L, a.Hq, kD, a.q_s, kBQ)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mk, a.k, a.B, a.L, a.Hkv, kD, a.k_s, kBK)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mv, a.v, a.B, a.L, a.Hkv, kD, a.v_s, kBK)) != cudaSuccess) return e;
-  if ((e = make_tma_bshd(&mdo, a.dout, a.B, a.L, a.Hq, kD, a.do_s, kBQ)) != cudaSuccess) return e;
-  const int64_t acc_s[3] = {static_cast<int64_t>(a.L) * a.Hq * kD, static_cast<int64_t>(a.Hq) * kD, kD};
-  if ((e = make_tma_bshd(&mdq, dq_acc, a.B, a.L, a.Hq, kD, acc_s, kBQ, 4)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mq, a.q, a.B, a.L, a.Hq, D, a.q_s, kBQ)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mk, a.k, a.B, a.L, a.Hkv, D, a.k_s, kBK)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mv, a.v, a.B, a.L, a.Hkv, D, a.v_s, kBK)) != cudaSuccess) return e;
+  if ((e = make_tma_bshd(&mdo, a.dout, a.B, a.L, a.Hq, D, a.do_s, kBQ)) != cudaSuccess) return e;
+  const int64_t acc_s[3] = {static_cast<int64_t>(a.L) * a.Hq * D, static_cast<int64_t>(a.Hq) * D, D};
+  if ((e = make_tma_bshd(&mdq, dq_acc, a.B, a.L, a.Hq, D, acc_s, kBQ, 4)) != cudaSuccess) return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   static int sm_count[64] = {};
@@ -626,12 +641,23 @@ cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_ac
   p.sl2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);
   p.lse_sb = a.lse_s[0];
   p.lse_sh = a.lse_s[1];
-  if ((e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)) !=
+  if ((e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes)) !=
       cudaSuccess)
     return e;
   const int grid = static_cast<int>(units < sms ? units : sms);
-  bwd_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+  bwd_tc_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float *dk_acc, float *dv_acc,
+                               cudaStream_t stream) {
+  switch (a.D) {
+    case 64: return launch_tc<64>(a, dsum, dq_acc, dk_acc, dv_acc, stream);
+    case 128: return launch_tc<128>(a, dsum, dq_acc, dk_acc, dv_acc, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace attnsink

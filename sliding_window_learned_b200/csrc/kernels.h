@@ -71,7 +71,7 @@ struct BwdArgs {
 };
 size_t bwd_workspace_bytes(const BwdArgs &a);
 cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream);
-// The tcgen05 main pass of the backward for D = 128: dQ, dK, dV summed in
+// The tcgen05 main pass of the backward (D = 64 or 128): dQ, dK, dV summed in
 // fp32 workspaces ([B, L, Hq, D], [B, L, Hkv, D], zeroed by the caller) from
 // Dsum ([B, Hq, L]).
 cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float *dk_acc, float *dv_acc,
