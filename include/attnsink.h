@@ -200,7 +200,8 @@ int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
  * a combine kernel merges only the chunks that exist, in chunk order, adding
  * the sink once.  The partials live in a workspace taken from a library-owned
  * stream-ordered memory pool (cudaMallocAsync/cudaFreeAsync on `stream`).
- * Supported: D in {64, 128, 256}, Hq/Hkv <= 16.
+ * Supported: D in {64, 128, 256}, Hq/Hkv <= 16 (<= 8 at D = 256; larger groups
+ * return ATTN_EUNSUPPORTED).
  */
 int attn_sink_decode(const attn_tensor *q, const attn_tensor *kcache,
                      const attn_tensor *vcache, const attn_tensor *seqlens,
