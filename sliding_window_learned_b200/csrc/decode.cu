@@ -186,11 +186,14 @@ struct DCfg {
   static_assert(!kF8 || D % 128 == 0, "FP8 rows are whole 128-byte chunks");
 };
 
-// Two e4m3 values (low byte first) to an f16 pair: one cvt, exact (every
-// e4m3 value, subnormals included, is a normal f16; NaN stays NaN).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
-  uint32_t h;
-  asm("{.reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t;}" : "=r"(h) : "r"(two_bytes));
+// Four e4m3 values (a 32-bit word, low byte first) to two f16 pairs: the word
+// splits into its 16-bit halves, one cvt each; exact (every e4m3 value,
+// subnormals included, is a normal f16; NaN stays NaN).
+__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t w) {
+  uint2 h;
+  asm("{.reg .b16 lo, hi; mov.b32 {lo, hi}, %2; cvt.rn.f16x2.e4m3x2 %0, lo; cvt.rn.f16x2.e4m3x2 %1, hi;}"
+      : "=r"(h.x), "=r"(h.y)
+      : "r"(w));
   return h;
 }
 
@@ -484,15 +487,10 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
             if (valid)
               x = *reinterpret_cast<const uint4 *>(src + kv * C::kTileBytes + c8 * C::kTK * 128 + row * 128 +
                                                    ((u ^ (row & 7)) << 4));
-            uint4 lo, hi;                          // elements 0..7 and 8..15 as f16
-            lo.x = e4m3x2_to_f16x2(x.x & 0xFFFFu);
-            lo.y = e4m3x2_to_f16x2(x.x >> 16);
-            lo.z = e4m3x2_to_f16x2(x.y & 0xFFFFu);
-            lo.w = e4m3x2_to_f16x2(x.y >> 16);
-            hi.x = e4m3x2_to_f16x2(x.z & 0xFFFFu);
-            hi.y = e4m3x2_to_f16x2(x.z >> 16);
-            hi.z = e4m3x2_to_f16x2(x.w & 0xFFFFu);
-            hi.w = e4m3x2_to_f16x2(x.w >> 16);
+            const uint2 a = e4m3x4_to_f16x4(x.x), b = e4m3x4_to_f16x4(x.y);
+            const uint2 c = e4m3x4_to_f16x4(x.z), d = e4m3x4_to_f16x4(x.w);
+            const uint4 lo = make_uint4(a.x, a.y, b.x, b.y);   // elements 0..7 as f16
+            const uint4 hi = make_uint4(c.x, c.y, d.x, d.y);   // elements 8..15
             const int col = c8 * 128 + u * 16;     // first element of this unit
             const int cb = col >> 6, ub = (col & 63) >> 3;
             uint8_t *drow = conv + kv * C::kBf16TileBytes + cb * C::kTK * 128 + row * 128;
