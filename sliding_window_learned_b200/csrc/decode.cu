@@ -147,42 +147,48 @@ struct StageInfo {
   int pad;
 };
 
-// kF8: the cache holds FP8 e4m3 bytes.  Its tiles arrive in 128-byte
-// (128-element) swizzled chunks; each consumer warp converts its 16 keys of K
-// and V to f16 (one cvt per pair, exact) into a tile of the 16-bit layout
-// (kConvBytes), and the MMA code below runs on that tile in f16: q is
-// converted to f16 after a power-of-two scale that puts its largest magnitude
-// in [2^13, 2^14) (undone in the softmax scale), and P is f16.
+// kF8: the cache holds FP8 e4m3 bytes, in 128-byte (128-element) swizzled
+// chunks.  Each consumer warp converts its K and V operands to f16 in
+// registers straight from the stage (one cvt per pair, exact) and runs the
+// MMAs below in f16: q is converted to f16 after a power-of-two scale that
+// puts its largest magnitude in [2^13, 2^14) (undone in the softmax scale),
+// and P is f16.  Because a 16-byte row unit read by ldmatrix hands each lane
+// four consecutive e4m3 values, the contraction index of S^T = K q^T is
+// permuted (k = 2t, 2t+1, 2t+8, 2t+9 of a k-step hold d = 4t .. 4t+3 of its
+// 16-d unit), and q is loaded in the same order; V is read as four 32-bit
+// words per lane (keys 2t, 2t+1, 2t+8, 2t+9; four consecutive d) and byte-
+// transposed, which permutes the d rows of O^T within each block of 32 (the
+// merge writes them back in order).
 // An FP8 cache delivers a key in half the bytes, so at D = 128 its tiles are
-// 192 keys for 12 consumer warps (three per SM sub-partition, to hide the
-// conversion's latency; 128 keys and 8 warps for groups of more than 8 heads,
-// whose accumulators need the registers); the merge buffer then lives in the
-// conversion tile (free at an item's end).
+// 192 keys for 12 consumer warps (128 keys and 8 warps for groups of more
+// than 8 heads, whose accumulators need the registers).  The merge at the end
+// of an item runs in the stage it has just consumed (one head tile per pass),
+// which is released after it; the ring takes all the rest of shared memory.
 template <int D, int NT, bool kF8>
 struct DCfg {
   static constexpr int kCW = (kF8 && D == 128) ? (NT == 1 ? 12 : 8) : kConsumerWarps;   // consumer warps
   static constexpr int kTK = 16 * kCW;                    // keys per tile
   static constexpr int kThreads = (kCW + 1) * 32;         // + the producer warp
-  static constexpr bool kMergeInConv = kF8;
+  static constexpr bool kMergeInStage = kF8;
+  static constexpr int kMergePasses = kMergeInStage ? NT : 1;   // head tiles merged one pass at a time
   static constexpr int kChunks = D / 64;                  // 64-element chunks of a bf16 row
   static constexpr int kChunks8 = D / 128;                // 128-element chunks of an FP8 row
   static constexpr int kTileBytes = kTK * D * (kF8 ? 1 : 2);   // one K (or V) tile as stored
-  static constexpr int kBf16TileBytes = kTK * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
-  static constexpr int kConvBytes = kF8 ? 2 * kBf16TileBytes : 0;
   static constexpr int kMergeBytes = kCW * NT * 8 * D * 4;
-  static constexpr int kRingBudget = (kF8 ? 221184 : 196608) - kConvBytes - (kMergeInConv ? 0 : kMergeBytes);
+  static constexpr int kRingBudget = kF8 ? 232448 - 1024 - 2048 : 196608 - kMergeBytes;
   static constexpr int kStages = (kRingBudget / kStageBytes) > 12 ? 12 : (kRingBudget / kStageBytes);
-  static constexpr int kConvOffset = kStages * kStageBytes;
-  static constexpr int kMergeOffset = kMergeInConv ? kConvOffset : kConvOffset + kConvBytes;
-  static constexpr int kInfoOffset = kConvOffset + kConvBytes + (kMergeInConv ? 0 : kMergeBytes);
-  static_assert(!kMergeInConv || kMergeBytes <= kConvBytes, "merge buffer fits the conversion tile");
+  static constexpr int kMergeOffset = kStages * kStageBytes;   // (16-bit cache only)
+  static constexpr int kInfoOffset = kStages * kStageBytes + (kMergeInStage ? 0 : kMergeBytes);
+  static_assert(!kMergeInStage || kCW * (NT / kMergePasses) * 8 * D * 4 <= kStageBytes,
+                "one merge pass fits a stage");
   // stage descriptors, full/empty barriers, per-warp (max, sum) for the merge,
   // the abort flag; plus 1 KB of slack for aligning the base to 1 KB
   static constexpr int kInfoBytes =
       (kStages * 32 + kStages * 16 + 2 * kCW * NT * 8 * 4 + 16 + 127) / 128 * 128;
   static constexpr int kSmemBytes = kInfoOffset + kInfoBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(!kF8 || kInfoBytes <= 2048, "FP8 ring budget leaves room for the stage info");
   static_assert(!kF8 || D % 128 == 0, "FP8 rows are whole 128-byte chunks");
 };
 
@@ -463,47 +469,8 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     const StageInfo si = info[s];
     if (si.flags & 4) break;
     const int key_w = warp * 16;  // this warp's 16 keys within the tile
-    uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
-    uint32_t vbase = kbase + C::kTileBytes;
-    if constexpr (kF8) {
-      // This warp's 16 K and V rows, e4m3 -> f16, into the conversion tile
-      // (the layout of a 16-bit stage); rows outside [nskip, nvalid) become
-      // zeros.  Then the FP8 stage goes back to the producer at once.
-      const uint8_t *src = smem + s * C::kStageBytes;
-      uint8_t *conv = smem + C::kConvOffset;
-      // lanes l and l + 16 share a row (one half each), so that the eight
-      // lanes of each 16-byte store phase cover eight rows: eight distinct
-      // swizzled slots, no bank conflict
-      const int row = key_w + (lane & 15);
-      const bool valid = row >= si.nskip && row < si.nvalid;
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-#pragma unroll
-        for (int c8 = 0; c8 < C::kChunks8; ++c8) {
-#pragma unroll
-          for (int uu = 0; uu < 4; ++uu) {
-            const int u = (lane >> 4) * 4 + uu;    // 16-byte unit (16 elements) of the 128-byte row
-            uint4 x = make_uint4(0, 0, 0, 0);
-            if (valid)
-              x = *reinterpret_cast<const uint4 *>(src + kv * C::kTileBytes + c8 * C::kTK * 128 + row * 128 +
-                                                   ((u ^ (row & 7)) << 4));
-            const uint2 a = e4m3x4_to_f16x4(x.x), b = e4m3x4_to_f16x4(x.y);
-            const uint2 c = e4m3x4_to_f16x4(x.z), d = e4m3x4_to_f16x4(x.w);
-            const uint4 lo = make_uint4(a.x, a.y, b.x, b.y);   // elements 0..7 as f16
-            const uint4 hi = make_uint4(c.x, c.y, d.x, d.y);   // elements 8..15
-            const int col = c8 * 128 + u * 16;     // first element of this unit
-            const int cb = col >> 6, ub = (col & 63) >> 3;
-            uint8_t *drow = conv + kv * C::kBf16TileBytes + cb * C::kTK * 128 + row * 128;
-            *reinterpret_cast<uint4 *>(drow + ((ub ^ (row & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4 *>(drow + (((ub + 1) ^ (row & 7)) << 4)) = hi;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      kbase = smem_u32(conv);
-      vbase = kbase + C::kBf16TileBytes;
-    }
+    const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
+    const uint32_t vbase = kbase + C::kTileBytes;
     if (si.flags & 1) {
       // first tile of a work item: load this kv head's grouped queries
 #pragma unroll
@@ -513,9 +480,12 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           const int hl = nt * 8 + g8;
           uint32_t x0 = 0, x1 = 0;
           if (hl < p.G) {
-            const __nv_bfloat16 *qr = p.q + si.b * p.q_sb + (si.hk * p.G + hl) * p.q_sh + kk * 16 + 2 * tig;
+            // 16-bit cache: k = 2t, 2t+1 | 2t+8, 2t+9 of the k-step are d =
+            // 16kk + 2t, +1 | +8, +9; FP8 cache: d = 16kk + 4t .. 4t+3
+            const __nv_bfloat16 *qr =
+                p.q + si.b * p.q_sb + (si.hk * p.G + hl) * p.q_sh + kk * 16 + (kF8 ? 4 : 2) * tig;
             x0 = *reinterpret_cast<const uint32_t *>(qr);
-            x1 = *reinterpret_cast<const uint32_t *>(qr + 8);
+            x1 = *reinterpret_cast<const uint32_t *>(qr + (kF8 ? 2 : 8));
           }
           qf[kk][nt][0] = x0;
           qf[kk][nt][1] = x1;
@@ -582,7 +552,31 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int f = 0; f < 4; ++f) sacc[nt][f] = 0.f;
-    {
+    if constexpr (kF8) {
+      // ldmatrix of e4m3 bytes: matrices (keys 0-7 | 8-15) x (unit u | u+1)
+      // of a 128-byte chunk; lane (g, t) receives d = 16u + 4t .. 4t+3 of
+      // keys g and g+8, i.e. the A fragments of k-steps u and u+1 once
+      // converted
+      const int r = lane & 7;
+      const int krow = key_w + r + ((lane >> 3) & 1) * 8;   // krow & 7 == r
+#pragma unroll
+      for (int c8 = 0; c8 < C::kChunks8; ++c8)
+#pragma unroll
+        for (int up = 0; up < 4; ++up) {
+          const int unit = 2 * up + (lane >> 4);
+          const uint32_t addr = kbase + c8 * (C::kTK * 128) + krow * 128 + ((unit ^ r) << 4);
+          uint32_t w0, w1, w2, w3;
+          ldmatrix_x4(addr, w0, w1, w2, w3);
+          const uint2 k0 = e4m3x4_to_f16x4(w0), k1 = e4m3x4_to_f16x4(w1);
+          const uint2 k2 = e4m3x4_to_f16x4(w2), k3 = e4m3x4_to_f16x4(w3);
+          const int kk = c8 * 8 + 2 * up;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_f16_16816(sacc[nt], k0.x, k1.x, k0.y, k1.y, qf[kk][nt][0], qf[kk][nt][1]);
+            mma_f16_16816(sacc[nt], k2.x, k3.x, k2.y, k3.y, qf[kk + 1][nt][0], qf[kk + 1][nt][1]);
+          }
+        }
+    } else {
       const int krow = key_w + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -591,12 +585,8 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4(addr, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if constexpr (kF8)
-            mma_f16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
-          else
-            mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
-        }
+        for (int nt = 0; nt < NT; ++nt)
+          mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
       }
     }
     // ---- online softmax per head (no sink here) ----
@@ -641,7 +631,43 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       pb[nt][1] = movmatrix_trans(kF8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3));
     }
     // ---- O^T[D x 8*NT] += V_w^T P^T ----
-    {
+    if constexpr (kF8) {
+      // Lane (g, t) reads d = 32j + 4g .. 4g+3 of keys 2t, 2t+1, 2t+8, 2t+9
+      // (one 32-bit word each; rows outside [nskip, nvalid) become zeros, as
+      // they may hold NaN bytes) and byte-transposes them into key pairs per
+      // d: O^T rows g and g+8 of m-tile 2j are d = 32j + 4g and 4g + 1, of
+      // m-tile 2j+1 d = 32j + 4g + 2 and 4g + 3.
+      const int ka = key_w + 2 * tig;
+      const bool va = ka >= si.nskip && ka < si.nvalid, vb = ka + 1 >= si.nskip && ka + 1 < si.nvalid;
+      const bool vc = ka + 8 >= si.nskip && ka + 8 < si.nvalid, vd = ka + 9 >= si.nskip && ka + 9 < si.nvalid;
+      const uint8_t *vt = smem + s * C::kStageBytes + C::kTileBytes;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const int bo = (j & 3) * 32 + 4 * g8;      // byte of d = 32j + 4g within its 128-byte chunk
+        const int unit = bo >> 4, wb = bo & 15;
+        const uint8_t *cb = vt + (j >> 2) * (C::kTK * 128) + wb;
+        // rows ka, ka+8 have (row & 7) == 2t; rows ka+1, ka+9 have 2t+1
+        const int sa = (unit ^ (2 * tig)) << 4, sb = (unit ^ (2 * tig + 1)) << 4;
+        uint32_t wa = *reinterpret_cast<const uint32_t *>(cb + ka * 128 + sa);
+        uint32_t wbb = *reinterpret_cast<const uint32_t *>(cb + (ka + 1) * 128 + sb);
+        uint32_t wc = *reinterpret_cast<const uint32_t *>(cb + (ka + 8) * 128 + sa);
+        uint32_t wd = *reinterpret_cast<const uint32_t *>(cb + (ka + 9) * 128 + sb);
+        wa = va ? wa : 0u;
+        wbb = vb ? wbb : 0u;
+        wc = vc ? wc : 0u;
+        wd = vd ? wd : 0u;
+        // (key 2t, key 2t+1) byte pairs of d0, d1 and of d2, d3; likewise 2t+8, 2t+9
+        const uint2 lo01 = e4m3x4_to_f16x4(__byte_perm(wa, wbb, 0x5140));
+        const uint2 lo23 = e4m3x4_to_f16x4(__byte_perm(wa, wbb, 0x7362));
+        const uint2 hi01 = e4m3x4_to_f16x4(__byte_perm(wc, wd, 0x5140));
+        const uint2 hi23 = e4m3x4_to_f16x4(__byte_perm(wc, wd, 0x7362));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_f16_16816(o[2 * j][nt], lo01.x, lo01.y, hi01.x, hi01.y, pb[nt][0], pb[nt][1]);
+          mma_f16_16816(o[2 * j + 1][nt], lo23.x, lo23.y, hi23.x, hi23.y, pb[nt][0], pb[nt][1]);
+        }
+      }
+    } else {
       const int vrow = key_w + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
       for (int dm = 0; dm < D / 16; ++dm) {
@@ -650,22 +676,20 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(addr, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if constexpr (kF8)
-            mma_f16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-          else
-            mma_bf16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-        }
+        for (int nt = 0; nt < NT; ++nt)
+          mma_bf16_16816(o[dm][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
       }
     }
     // release the stage (generic-proxy writes above are ordered before the
-    // next TMA write into it); an FP8 stage was released after conversion
+    // next TMA write into it); an FP8 stage is only read here, and the last
+    // one of an item is released after the merge that reuses it
     if constexpr (!kF8) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-    } else {
-      __syncwarp();   // the conversion tile is rewritten only after every lane's MMAs
+    } else if (!(si.flags & 2)) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
 
     if (si.flags & 2) {
@@ -679,7 +703,8 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
           l_run[nt][e] = l;
         }
-      named_barrier_sync(kBarMerge, C::kCW * 32);  // previous merge fully read
+      // previous merge fully read (FP8: and every warp done with this stage)
+      named_barrier_sync(kBarMerge, C::kCW * 32);
       if (g8 == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -689,41 +714,59 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
             merge_l[warp * NT * 8 + nt * 8 + 2 * tig + e] = l_run[nt][e];
           }
       }
-      float *mw = merge + warp * (NT * 8 * D);  // [head][d]
-#pragma unroll
-      for (int dm = 0; dm < D / 16; ++dm)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int hh = nt * 8 + 2 * tig;
-          mw[hh * D + dm * 16 + g8] = o[dm][nt][0];
-          mw[(hh + 1) * D + dm * 16 + g8] = o[dm][nt][1];
-          mw[hh * D + dm * 16 + g8 + 8] = o[dm][nt][2];
-          mw[(hh + 1) * D + dm * 16 + g8 + 8] = o[dm][nt][3];
-        }
-      named_barrier_sync(kBarMerge, C::kCW * 32);
+      // the per-warp O^T partials go through the merge buffer (FP8: the
+      // stage just consumed), kTP head tiles per pass
+      constexpr int kTP = NT / C::kMergePasses;
+      float *mbuf = C::kMergeInStage ? reinterpret_cast<float *>(smem + s * C::kStageBytes) : merge;
       const int tid = threadIdx.x;  // 0 .. consumer threads - 1
       const int gsplit = p.base[si.b] + si.split;
-      for (int e = tid; e < p.G * D; e += C::kCW * 32) {
-        const int hh = e / D, d = e - hh * D;
-        float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < C::kCW; ++w) M = fmaxf(M, merge_m[w * NT * 8 + hh]);
-        float num = 0.f, den = 0.f;
+      for (int ps = 0; ps < C::kMergePasses; ++ps) {
+        if (ps > 0) named_barrier_sync(kBarMerge, C::kCW * 32);   // previous pass fully read
+        float *mw = mbuf + warp * (kTP * 8 * D);  // [head of the pass][d]
 #pragma unroll
-        for (int w = 0; w < C::kCW; ++w) {
-          const float mw_ = merge_m[w * NT * 8 + hh];
-          const float f = (mw_ == -INFINITY) ? 0.f : ex2_approx(mw_ - M);
-          num += f * merge[w * (NT * 8 * D) + hh * D + d];
-          den += f * merge_l[w * NT * 8 + hh];
+        for (int dm = 0; dm < D / 16; ++dm)
+#pragma unroll
+          for (int j = 0; j < kTP; ++j) {
+            const int nt = ps * kTP + j;
+            const int hh = j * 8 + 2 * tig;
+            const int d0 = kF8 ? 32 * (dm >> 1) + 4 * g8 + 2 * (dm & 1) : dm * 16 + g8;  // O^T row g
+            const int d1 = kF8 ? d0 + 1 : d0 + 8;                                       // O^T row g + 8
+            mw[hh * D + d0] = o[dm][nt][0];
+            mw[(hh + 1) * D + d0] = o[dm][nt][1];
+            mw[hh * D + d1] = o[dm][nt][2];
+            mw[(hh + 1) * D + d1] = o[dm][nt][3];
+          }
+        named_barrier_sync(kBarMerge, C::kCW * 32);
+        const int h0 = ps * kTP * 8;
+        const int nh = min(p.G - h0, kTP * 8);
+        for (int e = tid; e < nh * D; e += C::kCW * 32) {
+          const int hl = e / D, d = e - hl * D, hh = h0 + hl;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < C::kCW; ++w) M = fmaxf(M, merge_m[w * NT * 8 + hh]);
+          float num = 0.f, den = 0.f;
+#pragma unroll
+          for (int w = 0; w < C::kCW; ++w) {
+            const float mw_ = merge_m[w * NT * 8 + hh];
+            const float f = (mw_ == -INFINITY) ? 0.f : ex2_approx(mw_ - M);
+            num += f * mbuf[w * (kTP * 8 * D) + hl * D + d];
+            den += f * merge_l[w * NT * 8 + hh];
+          }
+          const int hq = si.hk * p.G + hh;
+          const size_t row = static_cast<size_t>(gsplit) * p.Hq + hq;
+          p.o_part[row * D + d] = num / den * vdesc;
+          if (d == 0) p.lse_part[row] = (M + log2f(den)) * kLn2;
         }
-        const int hq = si.hk * p.G + hh;
-        const size_t row = static_cast<size_t>(gsplit) * p.Hq + hq;
-        p.o_part[row * D + d] = num / den * vdesc;
-        if (d == 0) p.lse_part[row] = (M + log2f(den)) * kLn2;
       }
-      // the merge buffer is the conversion tile: every reader is done before
-      // any warp converts the next tile into it
-      if constexpr (C::kMergeInConv) named_barrier_sync(kBarMerge, C::kCW * 32);
+      if constexpr (C::kMergeInStage) {
+        // every reader of the merge is done; its generic writes are ordered
+        // before the next TMA write into the stage
+        named_barrier_sync(kBarMerge, C::kCW * 32);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
     }
   }
 }
