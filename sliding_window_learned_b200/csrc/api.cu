@@ -596,8 +596,10 @@ int prep_decode_fp8(const attn_tensor *q, const attn_tensor *kcache, const attn_
       return fail(ATTN_EINVAL, "FP8 cache strides must be multiples of 16 elements");
   }
   if ((rc = prep_decode(q, &kc, &vc, seqlens, sinks, window, scale, 0, out, out_args, empty))) return rc;
-  out_args->chunk = (out_args->chunk + 127) / 128 * 128;   // whole 128-key FP8 tiles
+  // whole tiles per split, so that no tile reads into the next split's keys
   out_args->fp8 = true;
+  const int tile = decode_tile_keys(*out_args);
+  out_args->chunk = (out_args->chunk + tile - 1) / tile * tile;
   out_args->k_descale = static_cast<const float *>(k_descale->data);
   out_args->v_descale = static_cast<const float *>(v_descale->data);
   return ATTN_OK;

@@ -32,6 +32,8 @@
 // below that bound without tying up registers in fp32 FMA loops.
 #include <math.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -155,10 +157,10 @@ struct StageInfo {
 // and P is f16.  Because a 16-byte row unit read by ldmatrix hands each lane
 // four consecutive e4m3 values, the contraction index of S^T = K q^T is
 // permuted (k = 2t, 2t+1, 2t+8, 2t+9 of a k-step hold d = 4t .. 4t+3 of its
-// 16-d unit), and q is loaded in the same order; V is read as four 32-bit
-// words per lane (keys 2t, 2t+1, 2t+8, 2t+9; four consecutive d) and byte-
-// transposed, which permutes the d rows of O^T within each block of 32 (the
-// merge writes them back in order).
+// 16-d unit), and q is loaded in the same order; V goes through
+// ldmatrix.trans of byte pairs (keys 2t, 2t+1 at two consecutive d per lane)
+// and one byte permute, which orders the d rows of O^T within each 16-d unit
+// as 0, 2, .., 14 then 1, 3, .., 15 (the merge writes them back in order).
 // An FP8 cache delivers a key in half the bytes, so at D = 128 its tiles are
 // 192 keys for 12 consumer warps (128 keys and 8 warps for groups of more
 // than 8 heads, whose accumulators need the registers).  The merge at the end
@@ -632,41 +634,52 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     }
     // ---- O^T[D x 8*NT] += V_w^T P^T ----
     if constexpr (kF8) {
-      // Lane (g, t) reads d = 32j + 4g .. 4g+3 of keys 2t, 2t+1, 2t+8, 2t+9
-      // (one 32-bit word each; rows outside [nskip, nvalid) become zeros, as
-      // they may hold NaN bytes) and byte-transposes them into key pairs per
-      // d: O^T rows g and g+8 of m-tile 2j are d = 32j + 4g and 4g + 1, of
-      // m-tile 2j+1 d = 32j + 4g + 2 and 4g + 3.
-      const int ka = key_w + 2 * tig;
-      const bool va = ka >= si.nskip && ka < si.nvalid, vb = ka + 1 >= si.nskip && ka + 1 < si.nvalid;
-      const bool vc = ka + 8 >= si.nskip && ka + 8 < si.nvalid, vd = ka + 9 >= si.nskip && ka + 9 < si.nvalid;
-      const uint8_t *vt = smem + s * C::kStageBytes + C::kTileBytes;
-#pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        const int bo = (j & 3) * 32 + 4 * g8;      // byte of d = 32j + 4g within its 128-byte chunk
-        const int unit = bo >> 4, wb = bo & 15;
-        const uint8_t *cb = vt + (j >> 2) * (C::kTK * 128) + wb;
-        // rows ka, ka+8 have (row & 7) == 2t; rows ka+1, ka+9 have 2t+1
-        const int sa = (unit ^ (2 * tig)) << 4, sb = (unit ^ (2 * tig + 1)) << 4;
-        uint32_t wa = *reinterpret_cast<const uint32_t *>(cb + ka * 128 + sa);
-        uint32_t wbb = *reinterpret_cast<const uint32_t *>(cb + (ka + 1) * 128 + sb);
-        uint32_t wc = *reinterpret_cast<const uint32_t *>(cb + (ka + 8) * 128 + sa);
-        uint32_t wd = *reinterpret_cast<const uint32_t *>(cb + (ka + 9) * 128 + sb);
-        wa = va ? wa : 0u;
-        wbb = vb ? wbb : 0u;
-        wc = vc ? wc : 0u;
-        wd = vd ? wd : 0u;
-        // (key 2t, key 2t+1) byte pairs of d0, d1 and of d2, d3; likewise 2t+8, 2t+9
-        const uint2 lo01 = e4m3x4_to_f16x4(__byte_perm(wa, wbb, 0x5140));
-        const uint2 lo23 = e4m3x4_to_f16x4(__byte_perm(wa, wbb, 0x7362));
-        const uint2 hi01 = e4m3x4_to_f16x4(__byte_perm(wc, wd, 0x5140));
-        const uint2 hi23 = e4m3x4_to_f16x4(__byte_perm(wc, wd, 0x7362));
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_f16_16816(o[2 * j][nt], lo01.x, lo01.y, hi01.x, hi01.y, pb[nt][0], pb[nt][1]);
-          mma_f16_16816(o[2 * j + 1][nt], lo23.x, lo23.y, hi23.x, hi23.y, pb[nt][0], pb[nt][1]);
+      // ldmatrix.trans of e4m3 bytes taken as 16-bit pairs: matrices (keys
+      // 0-7 | 8-15) x (unit u | u+1); lane (g, t) receives keys 2t, 2t+1 (or
+      // 2t+8, 2t+9) at d = 16u + 2g and 2g + 1, which one byte permute turns
+      // into key pairs per d: O^T rows g and g+8 of m-tile u are d = 16u + 2g
+      // and 16u + 2g + 1.  Rows outside [nskip, nvalid) may hold NaN bytes:
+      // on the tiles that have any, they are zeroed in the registers.
+      const int r = lane & 7;
+      const int vrow = key_w + r + ((lane >> 3) & 1) * 8;   // vrow & 7 == r
+      auto pv = [&](auto masked) {
+        uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+        if constexpr (decltype(masked)::value) {
+          const int ka = key_w + 2 * tig;
+          auto ok = [&](int k) { return k >= si.nskip && k < si.nvalid; };
+          mlo = (ok(ka) ? 0x0000FFFFu : 0u) | (ok(ka + 1) ? 0xFFFF0000u : 0u);
+          mhi = (ok(ka + 8) ? 0x0000FFFFu : 0u) | (ok(ka + 9) ? 0xFFFF0000u : 0u);
         }
-      }
+#pragma unroll
+        for (int c8 = 0; c8 < C::kChunks8; ++c8)
+#pragma unroll
+          for (int up = 0; up < 4; ++up) {
+            const int unit = 2 * up + (lane >> 4);
+            const uint32_t addr = vbase + c8 * (C::kTK * 128) + vrow * 128 + ((unit ^ r) << 4);
+            uint32_t w0, w1, w2, w3;
+            ldmatrix_x4_trans(addr, w0, w1, w2, w3);
+            if constexpr (decltype(masked)::value) {
+              w0 &= mlo;
+              w1 &= mhi;
+              w2 &= mlo;
+              w3 &= mhi;
+            }
+            const uint2 v0 = e4m3x4_to_f16x4(__byte_perm(w0, 0u, 0x3120));
+            const uint2 v1 = e4m3x4_to_f16x4(__byte_perm(w1, 0u, 0x3120));
+            const uint2 v2 = e4m3x4_to_f16x4(__byte_perm(w2, 0u, 0x3120));
+            const uint2 v3 = e4m3x4_to_f16x4(__byte_perm(w3, 0u, 0x3120));
+            const int dm = c8 * 8 + 2 * up;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_f16_16816(o[dm][nt], v0.x, v0.y, v1.x, v1.y, pb[nt][0], pb[nt][1]);
+              mma_f16_16816(o[dm + 1][nt], v2.x, v2.y, v3.x, v3.y, pb[nt][0], pb[nt][1]);
+            }
+          }
+      };
+      if (si.nskip <= key_w && si.nvalid >= key_w + 16)
+        pv(std::false_type{});
+      else
+        pv(std::true_type{});
     } else {
       const int vrow = key_w + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
@@ -730,7 +743,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           for (int j = 0; j < kTP; ++j) {
             const int nt = ps * kTP + j;
             const int hh = j * 8 + 2 * tig;
-            const int d0 = kF8 ? 32 * (dm >> 1) + 4 * g8 + 2 * (dm & 1) : dm * 16 + g8;  // O^T row g
+            const int d0 = kF8 ? dm * 16 + 2 * g8 : dm * 16 + g8;  // O^T row g
             const int d1 = kF8 ? d0 + 1 : d0 + 8;                                       // O^T row g + 8
             mw[hh * D + d0] = o[dm][nt][0];
             mw[(hh + 1) * D + d0] = o[dm][nt][1];
@@ -918,6 +931,12 @@ int decode_max_splits_per_seq(const DecodeArgs &a) {
   // a paged cache's split range starts up to 63 keys before the window
   const long long vis = (a.W < a.Smax ? a.W : a.Smax) + (a.page > 0 ? kTK - 1 : 0);
   return static_cast<int>((vis + a.chunk - 1) / a.chunk);
+}
+
+int decode_tile_keys(const DecodeArgs &a) {
+  if (!a.fp8 || a.Hkv <= 0) return kTK;
+  if (a.D == 128) return a.Hq / a.Hkv <= 8 ? DCfg<128, 1, true>::kTK : DCfg<128, 2, true>::kTK;
+  return DCfg<256, 1, true>::kTK;
 }
 
 size_t decode_workspace_bytes(const DecodeArgs &a) { return ws_layout(a).total; }

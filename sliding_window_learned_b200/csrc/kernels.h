@@ -82,6 +82,9 @@ cudaError_t launch_bwd_main_tc(const BwdArgs &a, const float *dsum, float *dq_ac
 size_t decode_workspace_bytes(const DecodeArgs &a);
 // Upper bound on the number of splits of one sequence for these arguments.
 int decode_max_splits_per_seq(const DecodeArgs &a);
+// Keys per K/V tile of the split kernel that runs for these arguments (D, the
+// group size Hq/Hkv and the cache type fix it).
+int decode_tile_keys(const DecodeArgs &a);
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream);
 // Sets every entry of a [B, Hq] max-logit output to -inf.
