@@ -88,6 +88,10 @@ CASES = [  # B, MP, P, Hq, Hkv, D, W, seqlens, extra pages
     (3, 6, 64, 8, 2, 256, 1 << 30, [384, 100, 0], 2),
     (2, 12, 64, 6, 2, 256, 200, [700, 65], 5),
     (2, 2, 1024, 8, 2, 64, 513, [2048, 1500], 1),
+    # pages smaller than a tile at the other head dims and at 16 heads per kv head
+    (2, 24, 16, 8, 2, 64, 300, [380, 45], 2),
+    (2, 10, 32, 4, 1, 256, 1 << 30, [300, 17], 2),
+    (2, 16, 16, 32, 2, 128, 200, [250, 64], 2),
 ]
 
 
