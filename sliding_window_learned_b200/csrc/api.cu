@@ -279,13 +279,15 @@ uint64_t g_tma_tick = 0;
 std::mutex g_tma_mu;
 }  // namespace
 
-cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
-                          int64_t d0, const int64_t strides_el[3], int box_rows, int elem_bytes) {
-  typedef CUresult (*encode_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-  static encode_fn encode = nullptr;
+typedef CUresult (*tma_encode_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda); null if the driver does not provide it.
+static tma_encode_fn tma_encode() {
+  static tma_encode_fn encode = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
     void *fn = nullptr;
@@ -293,8 +295,41 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      encode = reinterpret_cast<encode_fn>(fn);
+      encode = reinterpret_cast<tma_encode_fn>(fn);
   });
+  return encode;
+}
+
+static bool tma_cache_get(const TmaKey &key, void *map_out) {
+  std::lock_guard<std::mutex> lk(g_tma_mu);
+  for (TmaEntry &e : g_tma_cache)
+    if (e.valid && e.key == key) {
+      e.used = ++g_tma_tick;
+      memcpy(map_out, &e.map, sizeof(CUtensorMap));
+      return true;
+    }
+  return false;
+}
+
+static void tma_cache_put(const TmaKey &key, const CUtensorMap &map) {
+  std::lock_guard<std::mutex> lk(g_tma_mu);
+  TmaEntry *victim = &g_tma_cache[0];
+  for (TmaEntry &e : g_tma_cache) {
+    if (!e.valid) {
+      victim = &e;
+      break;
+    }
+    if (e.used < victim->used) victim = &e;
+  }
+  victim->key = key;
+  memcpy(&victim->map, &map, sizeof(CUtensorMap));
+  victim->used = ++g_tma_tick;
+  victim->valid = true;
+}
+
+cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
+                          int64_t d0, const int64_t strides_el[3], int box_rows, int elem_bytes) {
+  const tma_encode_fn encode = tma_encode();
   if (!encode) return cudaErrorNotSupported;
   TmaKey key;
   key.base = base;
@@ -307,15 +342,7 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
   key.s[2] = strides_el[2];
   key.box = box_rows;
   key.elem = elem_bytes;
-  {
-    std::lock_guard<std::mutex> lk(g_tma_mu);
-    for (TmaEntry &e : g_tma_cache)
-      if (e.valid && e.key == key) {
-        e.used = ++g_tma_tick;
-        memcpy(map_out, &e.map, sizeof(CUtensorMap));
-        return cudaSuccess;
-      }
-  }
+  if (tma_cache_get(key, map_out)) return cudaSuccess;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
                               static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
   // byte strides of dims 1..3 (innermost first): head, position, batch
@@ -340,19 +367,42 @@ cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   memcpy(map_out, &map, sizeof(CUtensorMap));
-  std::lock_guard<std::mutex> lk(g_tma_mu);
-  TmaEntry *victim = &g_tma_cache[0];
-  for (TmaEntry &e : g_tma_cache) {
-    if (!e.valid) {
-      victim = &e;
-      break;
-    }
-    if (e.used < victim->used) victim = &e;
-  }
-  victim->key = key;
-  memcpy(&victim->map, &map, sizeof(CUtensorMap));
-  victim->used = ++g_tma_tick;
-  victim->valid = true;
+  tma_cache_put(key, map);
+  return cudaSuccess;
+}
+
+cudaError_t make_tma_pages5d(void *map_out, const void *base, int64_t npages, int64_t page, int64_t H,
+                             int64_t D, const int64_t strides_el[3]) {
+  const tma_encode_fn encode = tma_encode();
+  if (!encode) return cudaErrorNotSupported;
+  if (D % 64 != 0 || page < 1 || page > 256) return cudaErrorInvalidValue;
+  TmaKey key;
+  key.base = base;
+  key.d[0] = D;
+  key.d[1] = H;
+  key.d[2] = page;
+  key.d[3] = npages;
+  key.s[0] = strides_el[0];
+  key.s[1] = strides_el[1];
+  key.s[2] = strides_el[2];
+  key.box = static_cast<int>(page);
+  key.elem = -5;                     // (the 5-D page view; no 4-D map has this)
+  if (tma_cache_get(key, map_out)) return cudaSuccess;
+  const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(page), static_cast<cuuint64_t>(D / 64),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(npages)};
+  // byte strides of dims 1..4: position in page, chunk, head, page
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(strides_el[1]) * 2, 128,
+                                 static_cast<cuuint64_t>(strides_el[2]) * 2,
+                                 static_cast<cuuint64_t>(strides_el[0]) * 2};
+  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(page), static_cast<cuuint32_t>(D / 64), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  alignas(64) CUtensorMap map;
+  const CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  memcpy(map_out, &map, sizeof(CUtensorMap));
+  tma_cache_put(key, map);
   return cudaSuccess;
 }
 

@@ -10,8 +10,9 @@
 //   split    persistent: one work item = (split, kv head).  A TMA producer
 //            warp streams 64-key K/V tiles of that head into a ring of stages
 //            (for a paged cache, each tile from the pool page(s) the block
-//            table names: one box per tile, or 64/page boxes for pages of 16
-//            or 32 positions);
+//            table names: one box per tile, or for pages of 16 or 32
+//            positions one box per page holding every channel chunk, through
+//            a 5-D view of the pool);
 //            four consumer warps each take 16 keys of every tile and run
 //            S^T = K q^T and O^T += V^T P^T on the warp-level tensor cores
 //            (the Hq/Hkv grouped query heads are the N = 8 dimension), with an
@@ -138,6 +139,11 @@ struct SplitParams {
   const int *block_table;
   int64_t bt_s0;
   int page, page_shift, max_pages, align;
+  // log2 of the key rows R of one K (or V) TMA box: a 16-bit stage holds, per
+  // K/V tile, [box][64-channel chunk][row in box][128 bytes] (R = the tile's
+  // 64 rows, i.e. [chunk][row], except for pages of 16 or 32 positions, whose
+  // box is one page of every chunk)
+  int rows_shift;
   // FP8 e4m3 cache: per-kv-head dequantisation scales (key row = k_descale *
   // e4m3 row; v_descale scales the partial output)
   const float *k_descale, *v_descale;
@@ -346,10 +352,10 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
         }
       }
     }
-    // Pages smaller than a tile (several boxes per tile): the whole warp
+    // Pages smaller than a tile (several pages per tile): the whole warp
     // follows one control flow; lane 0 claims work, waits for free stages and
     // arms their barriers (results shared by shuffle), and the copies of a
-    // tile (one per page box, chunk and K/V) are issued by one lane each.
+    // tile (one per page and K/V) are issued by one lane each.
     if (small_pages) {
       if (lane == 0) {
         tma_prefetch_desc(&tmK);
@@ -424,22 +430,18 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
                 tma_load_4d(dst + C::kTileBytes + c * C::kTK * 128, &tmV, &full[s], c * 64, hk, key0, b);
               }
           } else {
-            // key0 is a multiple of 64 here, so each box of min(64, page) rows
-            // lies in one page.  A table entry outside the pool (or a page
-            // number past the table, for rows beyond the sequence end) loads
-            // zero rows: the box is out of range and filled, and it still
-            // delivers its bytes.  Lane (r, c, kv) issues box r's chunk c of
-            // K (kv = 0) or V (kv = 1).
-            const int rows = C::kTK / nbox;
-            const int copies = nbox * C::kChunks * 2;
-            const int r = lane / (C::kChunks * 2), c = (lane >> 1) % C::kChunks, kv = lane & 1;
+            // key0 is a multiple of 64 here, so the tile is nbox whole pages.
+            // Lane (r, kv) issues page r of K (kv = 0) or V (kv = 1): one box
+            // of every 64-channel chunk of the page's rows (5-D page view),
+            // at box slot r of the stage layout.  A table entry outside the
+            // pool (or a page number past the table, for rows beyond the
+            // sequence end) loads zero rows: the box is out of range and
+            // filled, and it still delivers its bytes.
+            const int r = lane >> 1, kv = lane & 1;
             const int blk_r = __shfl_sync(0xffffffffu, blk, r < nbox ? r : 0);
-            if (lane < copies) {
-              const int r0 = r * rows;
-              const int row_in_page = (key0 + r0) & (p.page - 1);
-              tma_load_4d(dst + kv * C::kTileBytes + c * C::kTK * 128 + r0 * 128, kv ? &tmV : &tmK, &full[s],
-                          c * 64, hk, row_in_page, blk_r);
-            }
+            if (lane < 2 * nbox)
+              tma_load_5d(dst + kv * C::kTileBytes + r * (C::kChunks * 128 * p.page), kv ? &tmV : &tmK,
+                          &full[s], 0, 0, 0, hk, blk_r);
           }
         }
       }
@@ -458,6 +460,19 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
   // ------------------------------------------------------------- consumers
   const int g8 = lane >> 2;       // mma "group" (row within an 8-row block)
   const int tig = lane & 3;       // thread in group
+  // 16-bit stage: byte offset of a key row within a K/V tile, and of a
+  // 64-channel chunk within a box ([box][chunk][row in box][128 bytes]; the
+  // row's swizzle phase stays row & 7, as a box holds a multiple of 8 rows)
+  const int rs = p.rows_shift;
+  auto row_off = [&](int row) -> uint32_t {
+    return static_cast<uint32_t>((((row >> rs) * C::kChunks) << (rs + 7)) + ((row & ((1 << rs) - 1)) << 7));
+  };
+  const uint32_t cstride = 128u << rs;
+  const int key_w = warp * 16;    // this warp's 16 keys within a tile
+  const int krow = key_w + (lane & 7) + ((lane >> 3) & 1) * 8;   // ldmatrix rows of S^T = K q^T
+  const int vrow = key_w + (lane & 7) + (lane >> 4) * 8;         // ldmatrix.trans rows of V^T
+  const uint32_t krow_off = row_off(krow), vrow_off = row_off(vrow);
+  const uint32_t zrow_off = row_off(key_w + (lane & 15));        // V rows zeroed by lanes l, l + 16
   float sl2 = p.scale_log2;       // (FP8: times the item's key descale)
   float vdesc = 1.f;              // (FP8: the item's value descale)
   uint32_t qf[D / 16][NT][2];     // B fragments of q^T, per k-step and head tile
@@ -470,7 +485,6 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     ++slot;
     const StageInfo si = info[s];
     if (si.flags & 4) break;
-    const int key_w = warp * 16;  // this warp's 16 keys within the tile
     const uint32_t kbase = smem_u32(smem + s * C::kStageBytes);
     const uint32_t vbase = kbase + C::kTileBytes;
     if (si.flags & 1) {
@@ -539,7 +553,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       const int kidx = key_w + (lane & 15);
       if (kidx >= si.nvalid || kidx < si.nskip) {
         for (int c = 0; c < C::kChunks; ++c) {
-          uint8_t *row = smem + s * C::kStageBytes + C::kTileBytes + c * C::kTK * 128 + kidx * 128;
+          uint8_t *row = smem + s * C::kStageBytes + C::kTileBytes + c * cstride + zrow_off;
           const int half = lane >> 4;
 #pragma unroll
           for (int u = 0; u < 4; ++u)
@@ -560,13 +574,13 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       // keys g and g+8, i.e. the A fragments of k-steps u and u+1 once
       // converted
       const int r = lane & 7;
-      const int krow = key_w + r + ((lane >> 3) & 1) * 8;   // krow & 7 == r
+      const int krow8 = key_w + r + ((lane >> 3) & 1) * 8;   // krow8 & 7 == r
 #pragma unroll
       for (int c8 = 0; c8 < C::kChunks8; ++c8)
 #pragma unroll
         for (int up = 0; up < 4; ++up) {
           const int unit = 2 * up + (lane >> 4);
-          const uint32_t addr = kbase + c8 * (C::kTK * 128) + krow * 128 + ((unit ^ r) << 4);
+          const uint32_t addr = kbase + c8 * (C::kTK * 128) + krow8 * 128 + ((unit ^ r) << 4);
           uint32_t w0, w1, w2, w3;
           ldmatrix_x4(addr, w0, w1, w2, w3);
           const uint2 k0 = e4m3x4_to_f16x4(w0), k1 = e4m3x4_to_f16x4(w1);
@@ -579,11 +593,10 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           }
         }
     } else {
-      const int krow = key_w + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const int unit = 2 * (kk & 3) + (lane >> 4);
-        const uint32_t addr = kbase + (kk >> 2) * (C::kTK * 128) + krow * 128 + ((unit ^ (krow & 7)) << 4);
+        const uint32_t addr = kbase + (kk >> 2) * cstride + krow_off + ((unit ^ (krow & 7)) << 4);
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4(addr, a0, a1, a2, a3);
 #pragma unroll
@@ -641,7 +654,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       // and 16u + 2g + 1.  Rows outside [nskip, nvalid) may hold NaN bytes:
       // on the tiles that have any, they are zeroed in the registers.
       const int r = lane & 7;
-      const int vrow = key_w + r + ((lane >> 3) & 1) * 8;   // vrow & 7 == r
+      const int vrow8 = key_w + r + ((lane >> 3) & 1) * 8;   // vrow8 & 7 == r
       auto pv = [&](auto masked) {
         uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
         if constexpr (decltype(masked)::value) {
@@ -655,7 +668,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
 #pragma unroll
           for (int up = 0; up < 4; ++up) {
             const int unit = 2 * up + (lane >> 4);
-            const uint32_t addr = vbase + c8 * (C::kTK * 128) + vrow * 128 + ((unit ^ r) << 4);
+            const uint32_t addr = vbase + c8 * (C::kTK * 128) + vrow8 * 128 + ((unit ^ r) << 4);
             uint32_t w0, w1, w2, w3;
             ldmatrix_x4_trans(addr, w0, w1, w2, w3);
             if constexpr (decltype(masked)::value) {
@@ -681,11 +694,10 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       else
         pv(std::true_type{});
     } else {
-      const int vrow = key_w + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
       for (int dm = 0; dm < D / 16; ++dm) {
         const int unit = 2 * (dm & 3) + ((lane >> 3) & 1);
-        const uint32_t addr = vbase + (dm >> 2) * (C::kTK * 128) + vrow * 128 + ((unit ^ (vrow & 7)) << 4);
+        const uint32_t addr = vbase + (dm >> 2) * cstride + vrow_off + ((unit ^ (vrow & 7)) << 4);
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(addr, a0, a1, a2, a3);
 #pragma unroll
@@ -866,10 +878,13 @@ cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cu
   } else if (a.page == 0) {
     if ((e = make_tma_bshd(&mk, a.kc, a.B, a.Smax, a.Hkv, D, a.kc_s, C::kTK)) != cudaSuccess) return e;
     if ((e = make_tma_bshd(&mv, a.vc, a.B, a.Smax, a.Hkv, D, a.vc_s, C::kTK)) != cudaSuccess) return e;
+  } else if (a.page < C::kTK) {
+    // one box per page (every chunk): the 5-D page view
+    if ((e = make_tma_pages5d(&mk, a.kc, a.npages, a.page, a.Hkv, D, a.kc_s)) != cudaSuccess) return e;
+    if ((e = make_tma_pages5d(&mv, a.vc, a.npages, a.page, a.Hkv, D, a.vc_s)) != cudaSuccess) return e;
   } else {
-    const int rows = a.page < C::kTK ? a.page : C::kTK;
-    if ((e = make_tma_bshd(&mk, a.kc, a.npages, a.page, a.Hkv, D, a.kc_s, rows)) != cudaSuccess) return e;
-    if ((e = make_tma_bshd(&mv, a.vc, a.npages, a.page, a.Hkv, D, a.vc_s, rows)) != cudaSuccess) return e;
+    if ((e = make_tma_bshd(&mk, a.kc, a.npages, a.page, a.Hkv, D, a.kc_s, C::kTK)) != cudaSuccess) return e;
+    if ((e = make_tma_bshd(&mv, a.vc, a.npages, a.page, a.Hkv, D, a.vc_s, C::kTK)) != cudaSuccess) return e;
   }
   SplitParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -898,6 +913,11 @@ cudaError_t launch_split(const DecodeArgs &a, const WsLayout &w, uint8_t *ws, cu
   while (a.page > 0 && (1 << p.page_shift) < a.page) ++p.page_shift;
   p.max_pages = a.max_pages;
   p.align = a.page > 0 ? C::kTK : 1;
+  p.rows_shift = 0;
+  if (!kF8) {
+    const int rows = (a.page != 0 && a.page < C::kTK) ? a.page : C::kTK;
+    while ((1 << p.rows_shift) < rows) ++p.rows_shift;
+  }
   p.k_descale = a.k_descale;
   p.v_descale = a.v_descale;
   int dev = 0, sms = 0;

@@ -102,5 +102,13 @@ cudaError_t launch_decode(const DecodeArgs &a, void *workspace, cudaStream_t str
 // ({d0, 1, box_rows, 1}, d0 <= 256, no swizzle), for bulk reductions.
 cudaError_t make_tma_bshd(void *map_out, const void *base, int64_t d3, int64_t d2, int64_t d1,
                           int64_t d0, const int64_t strides_el[3], int box_rows, int elem_bytes = 2);
+// TMA descriptor of a bf16 page pool [npages, page, H, D] (element strides of
+// the first three dimensions in strides_el; the last one contiguous) as 5-D
+// (64 channels, position in page, 64-channel chunk, head, page) with 128-byte
+// swizzle, whose box {64, page, D/64, 1, 1} is one page of one head, every
+// chunk: in shared memory [chunk][position][128 bytes].  D a multiple of 64,
+// page <= 256.  Returns cudaErrorInvalidValue if the driver rejects it.
+cudaError_t make_tma_pages5d(void *map_out, const void *base, int64_t npages, int64_t page, int64_t H,
+                             int64_t D, const int64_t strides_el[3]);
 
 }  // namespace attnsink
