@@ -169,3 +169,23 @@ def test_paged_decode_workload_sampled():
         ref = oracle.decode(inputs.bits(y["q"][b:b + 1]), inputs.bits(kb), inputs.bits(vb),
                             np.array([n], np.int32), y["sinks"].cpu().numpy(), cfg.W, cfg.scale)[0]
         _check(o[b:b + 1], ref, f"paged decode seq {b} (n={n})")
+
+
+@pytest.mark.parametrize("P", [16, 32, 64])
+def test_paged_strided_pools(P):
+    """K and V pages interleaved in one buffer [NB, P, 2, Hkv, D] (the pools are
+    strided slices of it): the tensor maps take the caller's strides, so the
+    output equals that of contiguous pools bit for bit, and the oracle's."""
+    B, MP, Hq, Hkv, D, W = 2, 128 // P * 3, 8, 2, 128, 200
+    q, kp, vp, table, sl, s = _paged_case(B, MP, P, Hq, Hkv, D, W, [300, 97], 2, seed=P + 5)
+    scale = 1.0 / np.sqrt(D)
+    buf = torch.stack([kp, vp], dim=2).to(DEV)          # [NB, P, 2, Hkv, D]
+    ks, vs = buf[:, :, 0], buf[:, :, 1]
+    assert ks.stride()[:3] == (P * 2 * Hkv * D, 2 * Hkv * D, D)
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=DEV)
+    swl.attn_sink_decode_paged(q.to(DEV), ks, vs, table.to(DEV), sl.to(DEV), s.to(DEV), W, scale, out)
+    torch.cuda.synchronize()
+    assert swl.attn_sink_get_status() == 0
+    o = out.float().cpu().numpy()
+    assert np.array_equal(o, _gpu(q, kp, vp, table, sl, s, W, scale))
+    _check(o, _oracle(q, kp, vp, table, sl, s, W, scale), f"strided pools P={P}")
