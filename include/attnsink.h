@@ -266,10 +266,12 @@ int attn_sink_decode_paged(const attn_tensor *q, const attn_tensor *kpages,
  *   seqlens, sinks, window, scale, out: as for attn_sink_decode.
  *
  * The same three launches as attn_sink_decode; the split kernel streams the
- * e4m3 tiles (half the bytes of bf16), each consumer warp converts its keys
- * to bf16 in shared memory (exact: every e4m3 value is a bf16 value) and the
- * key descale is folded into the softmax scale.  D in {128, 256}; Hq/Hkv as
- * for attn_sink_decode.
+ * e4m3 tiles (half the bytes of bf16), and each consumer warp converts its
+ * keys and values to f16 in registers as it feeds them to the tensor cores
+ * (exact: every e4m3 value is a normal f16 value); q enters in f16 under a
+ * power-of-two scale, P in f16, and the key descale is folded into the
+ * softmax scale, the value descale into the output scale.  D in {128, 256};
+ * Hq/Hkv as for attn_sink_decode.
  */
 int attn_sink_decode_fp8(const attn_tensor *q, const attn_tensor *kcache,
                          const attn_tensor *vcache, const attn_tensor *k_descale,
