@@ -6,7 +6,9 @@ captures (Nsight Compute) of a single kernel on a bounded device footprint.
   python -m sliding_window_learned_b200.ncu_driver --op bwd --workload prefill --launches 2
 
 (--op bwd runs one forward for O and LSE, then the backward passes; --op
-decode_fp8 quantises the workload's cache to e4m3 per kv head first.)
+decode_fp8 quantises the workload's cache to e4m3 per kv head first; --op
+decode_paged copies the cache into pools of --page positions at random pool
+positions, addressed through a block table.)
 
 It prints no timings (numbers taken under a profiler are not measurements);
 it exits non-zero if the device reports an error.
@@ -34,9 +36,10 @@ WORKLOADS = {
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["fwd", "decode", "bwd", "decode_fp8"], required=True)
+    ap.add_argument("--op", choices=["fwd", "decode", "bwd", "decode_fp8", "decode_paged"], required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--page", type=int, default=16, help="positions per page (--op decode_paged)")
     a = ap.parse_args(argv)
     build.build()
     dev = torch.device("cuda", 0)
@@ -77,6 +80,19 @@ def main(argv=None) -> int:
                     dst[:, :, hk] = (xs / d[hk]).to(torch.float8_e4m3fn)
             for _ in range(a.launches):
                 abi.attn_sink_decode_fp8(y["q"], k8, v8, kd, vd, y["seqlens"], y["sinks"], cfg.W, cfg.scale, out)
+        elif a.op == "decode_paged":
+            P = a.page
+            n_pages = cfg.B * (cfg.Smax // P)
+            perm = torch.randperm(n_pages, generator=torch.Generator(device=dev).manual_seed(0), device=dev)
+            kpool = torch.empty((n_pages, P, cfg.Hkv, cfg.D), dtype=torch.bfloat16, device=dev)
+            kpool[perm] = y["kcache"].reshape(n_pages, P, cfg.Hkv, cfg.D)
+            vpool = torch.empty_like(kpool)
+            vpool[perm] = y["vcache"].reshape(n_pages, P, cfg.Hkv, cfg.D)
+            table = perm.reshape(cfg.B, cfg.Smax // P).to(torch.int32)
+            del y["kcache"], y["vcache"]
+            for _ in range(a.launches):
+                abi.attn_sink_decode_paged(y["q"], kpool, vpool, table, y["seqlens"], y["sinks"], cfg.W,
+                                           cfg.scale, out)
         else:
             for _ in range(a.launches):
                 abi.attn_sink_decode(y["q"], y["kcache"], y["vcache"], y["seqlens"], y["sinks"],
