@@ -482,6 +482,9 @@ def run_ours(args, rank, world, local_rank):
         "decode_fp8": {"value": round(aggregate_rate(Kp * dbytes8, world, t_fp8) / 1e9, 2), "unit": "GB/s",
                        "ms_per_call": round(t_fp8 / Kp * 1e3, 4),
                        "frac": round(dbytes8 / (t_fp8 / Kp) / 1e9 / hbm_peak, 4),
+                       "traffic": profiled_traffic("decode_split_fp8", [
+                           "sliding_window_learned_b200/csrc/decode.cu",
+                           "sliding_window_learned_b200/csrc/ptx.cuh"]),
                        "what": "attn_sink_decode_fp8 on the decode workload, cache quantised to e4m3 per "
                                "kv head (bytes counted at one per element)"},
         "fwd_varlen": {"value": round(aggregate_rate(Kv * vl_flops, world, t_varlen) / 1e12, 3), "unit": "TFLOP/s",
