@@ -14,11 +14,13 @@ pool positions, attn_sink_decode_paged) is timed as `decode_paged`, the decode
 over the cache quantised to e4m3 (attn_sink_decode_fp8) as `decode_fp8`, the
 forward over a seeded mix of 24 packed sequences (attn_sink_fwd_varlen) as
 `fwd_varlen`, and the backward pass on the prefill workload (attn_sink_bwd) as
-`bwd`.
+`bwd`.  `workloads` times attn_sink_fwd on each prefill workload on its own
+(tiny, prefill, long causal, sink stress), each with its own clock record.
 `--impl reference` times
 the fp64 CPU oracle on a bounded sample of the same prefill workload.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       python bench.py --profile OP --workload NAME [--launches N]   (profiler driver)
 (N > 1: launch under torchrun; each rank runs its own copy of the workloads.)
 """
 from __future__ import annotations
@@ -42,6 +44,7 @@ from sliding_window_learned_b200 import inputs  # noqa: E402
 
 METRIC = "attn fwd TFLOP/s (useful) & % bf16 tensor peak; decode HBM GB/s & % of peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 8000.0
 
 
 def useful_fwd_flops(cfg) -> float:
@@ -89,17 +92,57 @@ def profiled_traffic(kernel: str, sources: list[str]):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clock, power and clock-event reasons sampled during a timed region.
 
+    NVML is polled from a background thread about once a millisecond (the
+    device is found by the PCI bus id torch reports, so CUDA_VISIBLE_DEVICES
+    does not matter); without NVML, nvidia-smi is sampled every 50 ms.  Only
+    readings are taken: no clock, power or other setting is changed."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.proc = None
         self.idx = device_index
+        self.proc = None
+        self.thread = None
+        self.nv = None
+        self.handle = None
+        self.samples = []
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(device_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nv = pynvml
+        except Exception:  # noqa: BLE001 - any NVML problem: fall back to nvidia-smi
+            self.nv = None
+
+    def _poll(self):
+        nv, h = self.nv, self.handle
+        while not self._stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), pw, int(rs)))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.001)
 
     def start(self):
+        self.samples = []
+        if self.nv is not None:
+            import threading
+            self._stop = False
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -109,6 +152,18 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self._stop = True
+            self.thread.join()
+            self.thread = None
+            if not self.samples:
+                return None
+            mx = float(self.nv.nvmlDeviceGetMaxClockInfo(self.handle, self.nv.NVML_CLOCK_SM))
+            reasons = sorted({nm for _, _, r in self.samples for bit, nm in self.REASONS.items() if r & bit})
+            sm = [x for x, _, _ in self.samples]
+            return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": mx,
+                    "power_w_max": round(max(p for _, p, _ in self.samples), 1),
+                    "samples": len(sm), "reasons": reasons, "source": "nvml, ~1 ms"}
         if self.proc is None:
             return None
         time.sleep(0.25)
@@ -135,7 +190,52 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
-                "reasons": sorted(reasons)}
+                "reasons": sorted(reasons), "source": "nvidia-smi, 50 ms"}
+
+
+def page_cache(y, cfg, page, seed, dev):
+    """The decode workload's cache copied into pools of `page` positions at
+    random pool positions; returns (kpool, vpool, block_table)."""
+    import torch
+    n_pages = cfg.B * (cfg.Smax // page)
+    perm = torch.randperm(n_pages, generator=torch.Generator(device=dev).manual_seed(seed), device=dev)
+    kpool = torch.empty((n_pages, page, cfg.Hkv, cfg.D), dtype=torch.bfloat16, device=dev)
+    kpool[perm] = y["kcache"].reshape(n_pages, page, cfg.Hkv, cfg.D)
+    vpool = torch.empty_like(kpool)
+    vpool[perm] = y["vcache"].reshape(n_pages, page, cfg.Hkv, cfg.D)
+    return kpool, vpool, perm.reshape(cfg.B, cfg.Smax // page).to(torch.int32)
+
+
+def quantise_e4m3(y, cfg, dev):
+    """The decode workload's cache quantised to e4m3 with one descale per kv
+    head (max |x| / 448); returns (k8, v8, k_descale, v_descale)."""
+    import torch
+    kd = torch.empty(cfg.Hkv, device=dev)
+    vd = torch.empty(cfg.Hkv, device=dev)
+    k8 = torch.empty(y["kcache"].shape, dtype=torch.float8_e4m3fn, device=dev)
+    v8 = torch.empty_like(k8)
+    for hk in range(cfg.Hkv):
+        for src, dst, d in ((y["kcache"], k8, kd), (y["vcache"], v8, vd)):
+            xs = src[:, :, hk].float()
+            d[hk] = torch.nan_to_num(xs, nan=0.0).abs().amax() / 448.0
+            dst[:, :, hk] = (xs / d[hk]).to(torch.float8_e4m3fn)
+            del xs
+    return k8, v8, kd, vd
+
+
+def forward_leg_report(cfg, launches, seconds, clk, nsets, world, peak, peak_src):
+    """One prefill workload timed on its own: useful TFLOP/s over all ranks,
+    time per launch, fraction of the measured bf16 peak, and its clocks."""
+    flops = useful_fwd_flops(cfg)
+    per = seconds / launches
+    return {"workload": cfg.name, "value": round(aggregate_rate(launches * flops, world, seconds) / 1e12, 3),
+            "unit": "TFLOP/s", "launches": launches, "ms_per_call": round(per * 1e3, 5),
+            "flops_per_launch": flops,
+            "frac": round(flops / per / 1e12 / peak, 4), "peak": peak, "peak_source": f"{peak_src} bf16 (burst)",
+            "l2": ("flushed before each launch (per-launch events)" if cfg.L <= 1024 else
+                   f"back-to-back launches over {nsets} input set(s), each launch's q, k, v, O "
+                   "(plus the other set's) larger than L2"),
+            "clocks": clk}
 
 
 # --------------------------------------------------------------- our arm
@@ -309,14 +409,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- the same decode over a paged cache (256-position pages at random
     # pool positions, addressed through a block table) ----
     page = 256
-    n_pages = dcfg.B * (dcfg.Smax // page)
-    perm = torch.randperm(n_pages, generator=torch.Generator(device=dev).manual_seed(rank), device=dev)
-    kpool = torch.empty((n_pages, page, dcfg.Hkv, dcfg.D), dtype=torch.bfloat16, device=dev)
-    kpool[perm] = y["kcache"].reshape(n_pages, page, dcfg.Hkv, dcfg.D)
-    vpool = torch.empty_like(kpool)
-    vpool[perm] = y["vcache"].reshape(n_pages, page, dcfg.Hkv, dcfg.D)
-    table = perm.reshape(dcfg.B, dcfg.Smax // page).to(torch.int32)
-    del perm
+    kpool, vpool, table = page_cache(y, dcfg, page, rank, dev)
 
     def dec_paged():
         swl.attn_sink_decode_paged(y["q"], kpool, vpool, table, y["seqlens"], y["sinks"], dcfg.W,
@@ -337,16 +430,7 @@ def run_ours(args, rank, world, local_rank):
     del kpool, vpool, table
 
     # ---- the same decode over its cache quantised to FP8 e4m3 per kv head ----
-    kdesc = torch.empty(dcfg.Hkv, device=dev)
-    vdesc = torch.empty(dcfg.Hkv, device=dev)
-    k8 = torch.empty(y["kcache"].shape, dtype=torch.float8_e4m3fn, device=dev)
-    v8 = torch.empty_like(k8)
-    for hk in range(dcfg.Hkv):
-        for src, dst, dsc in ((y["kcache"], k8, kdesc), (y["vcache"], v8, vdesc)):
-            xs = src[:, :, hk].float()
-            dsc[hk] = torch.nan_to_num(xs, nan=0.0).abs().amax() / 448.0
-            dst[:, :, hk] = (xs / dsc[hk]).to(torch.float8_e4m3fn)
-            del xs
+    k8, v8, kdesc, vdesc = quantise_e4m3(y, dcfg, dev)
 
     def dec_fp8():
         swl.attn_sink_decode_fp8(y["q"], k8, v8, kdesc, vdesc, y["seqlens"], y["sinks"], dcfg.W,
@@ -428,6 +512,66 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device status error in the backward pass")
     del bdo, bdq, bdk, bdv
 
+    # ---- every prefill workload on its own: back-to-back launches with
+    # their own clock record.  Two input sets alternate when one set (q, k, v,
+    # O) is smaller than twice L2, so that a launch never finds its inputs left
+    # in L2 by the previous launch; the tiny workload (launch-bound) is timed
+    # per launch with L2 flushed before each. ----
+    def forward_leg(cfg, launches, seed):
+        one = (cfg.B * cfg.L * (2 * cfg.Hq + 2 * cfg.Hkv) * cfg.D * 2)
+        nsets = 1 if one >= 256 * 1024 * 1024 else 2
+        sets = []
+        for si in range(nsets):
+            xs = inputs.make_prefill(cfg, seed=seed + si)
+            sets.append((xs["q"].to(dev), xs["k"].to(dev), xs["v"].to(dev), xs["sinks"].to(dev),
+                         torch.empty(xs["q"].shape, dtype=torch.bfloat16, device=dev),
+                         torch.empty(cfg.B, cfg.Hq, cfg.L, dtype=torch.float32, device=dev)))
+            del xs
+
+        def call(i):
+            a = sets[i % nsets]
+            swl.attn_sink_fwd(a[0], a[1], a[2], a[3], cfg.W, cfg.scale, a[4], a[5], stream)
+
+        for i in range(5):
+            call(i)
+        torch.cuda.synchronize()
+        per_launch = cfg.L <= 1024
+        sampler = ClockSampler(local_rank)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        sampler.start()
+        if per_launch:
+            tl = 0.0
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(launches)]
+            for i in range(launches):
+                flush.fill_(1.0)
+                evs[i][0].record(stream)
+                call(i)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            tl = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+        else:
+            e0.record(stream)
+            for i in range(launches):
+                call(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tl = e0.elapsed_time(e1) / 1e3
+        clk_leg = sampler.stop()
+        if swl.attn_sink_get_status() != 0:
+            raise RuntimeError(f"device status error in the {cfg.name} leg")
+        del sets
+        return tl, clk_leg, nsets
+
+    leg_specs = [("tiny", inputs.TINY, 200), ("prefill", inputs.PREFILL, 1000),
+                 ("long_causal", inputs.LONG_CAUSAL, 100), ("stress", inputs.STRESS, 1000)]
+    leg_raw = {}
+    for nm, cfg_l, n_l in leg_specs:
+        leg_raw[nm] = (cfg_l, n_l) + forward_leg(cfg_l, n_l, 3000 + 10 * rank)
+    leg_times = max_over_ranks([leg_raw[nm][2] for nm, _, _ in leg_specs], world, dev)
+
     # ---- max over ranks ----
     t_fwd, t_dec, t_all, t_e2e, t_e2e_serial, t_paged, t_varlen, t_fp8, t_bwd = max_over_ranks(
         [t_fwd, t_dec, t_all, t_e2e, t_e2e_serial, t_paged, t_varlen, t_fp8, t_bwd], world, dev)
@@ -470,7 +614,11 @@ def run_ours(args, rank, world, local_rank):
                    "roofline": {"kernel": "plan + split + combine", "bound": "hbm",
                                 "achieved": round(achieved_dec, 2), "peak": hbm_peak, "unit": "GB/s",
                                 "frac": round(achieved_dec / hbm_peak, 4),
-                                "peak_source": f"{peak_src} copy bandwidth",
+                                "peak_source": f"{peak_src} copy bandwidth (read + write)",
+                                "frac_of_nominal": round(achieved_dec / NOMINAL_HBM_GBS, 4),
+                                "note": "the decode only reads; the copy benchmark's read+write "
+                                        "figure can be exceeded, so frac_of_nominal (8 TB/s) is "
+                                        "given beside it",
                                 "traffic": profiled_traffic("decode_split", [
                                     "sliding_window_learned_b200/csrc/decode.cu",
                                     "sliding_window_learned_b200/csrc/ptx.cuh"])}},
@@ -508,6 +656,9 @@ def run_ours(args, rank, world, local_rank):
                         "step; the copies of neighbouring steps overlap the forward (input copies, "
                         "forward and output copies on three streams, two sets of device buffers); "
                         "serial_value: one step at a time on one stream"},
+        "workloads": {nm: forward_leg_report(leg_raw[nm][0], leg_raw[nm][1], tl_, leg_raw[nm][3],
+                                            leg_raw[nm][4], world, bf16_peak, peak_src)
+                      for (nm, _, _), tl_ in zip(leg_specs, leg_times)},
         "gpu_launches": K * 4,
         "clocks": clk,
         "timed_region_ms": round(t_all * 1e3, 3),
@@ -645,6 +796,81 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------- profiler driver
+def _profile_workloads():
+    return {
+        "tiny": inputs.TINY,
+        "prefill": inputs.PREFILL,
+        "long-causal": inputs.LONG_CAUSAL,
+        "stress": inputs.STRESS,
+        "decode": inputs.DECODE,
+        # same length distribution as the decode workload, 8 sequences (~1 GB of cache)
+        "decode-small": inputs.Decode("decode-small B8 Hq32 Hkv4 D128 n~U[4096,131072]", 8, 32, 4,
+                                      128, 131072, 4096, 131072, 131072),
+    }
+
+
+def run_profile(args) -> int:
+    """A few launches of one operation on one workload, for Nsight Compute
+    captures of a single kernel on a bounded device footprint.  It prints no
+    timings (numbers taken under a profiler are not measurements) and exits
+    non-zero if the device reports an error.
+
+    --profile bwd runs one forward for O and LSE, then the backward passes;
+    --profile decode_fp8 quantises the workload's cache to e4m3 per kv head
+    first; --profile decode_paged copies the cache into pools of --page
+    positions at random pool positions, addressed through a block table."""
+    import torch
+
+    from sliding_window_learned_b200 import abi, build
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = _profile_workloads()[args.workload]
+    op, n = args.profile, args.launches
+    if op in ("fwd", "bwd"):
+        if not isinstance(cfg, inputs.Prefill):
+            raise SystemExit(f"{op} needs a prefill workload")
+        x = inputs.make_prefill(cfg, seed=0, device=dev)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty(cfg.B, cfg.Hq, cfg.L, dtype=torch.float32, device=dev)
+        if op == "fwd":
+            for _ in range(n):
+                abi.attn_sink_fwd(x["q"], x["k"], x["v"], x["sinks"], cfg.W, cfg.scale, out, lse)
+        else:
+            abi.attn_sink_fwd(x["q"], x["k"], x["v"], x["sinks"], cfg.W, cfg.scale, out, lse)
+            g = torch.Generator(device=dev).manual_seed(1)
+            dout = torch.randn(x["q"].shape, device=dev, generator=g).to(torch.bfloat16)
+            dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+            dsink = torch.empty(cfg.Hq, dtype=torch.float32, device=dev)
+            for _ in range(n):
+                abi.attn_sink_bwd(x["q"], x["k"], x["v"], out, lse, dout, x["sinks"], cfg.W, cfg.scale,
+                                  dq, dk, dv, dsink)
+    else:
+        if not isinstance(cfg, inputs.Decode):
+            raise SystemExit("decode needs a decode workload")
+        y = inputs.make_decode(cfg, seed=0, device=dev)
+        out = torch.empty_like(y["q"])
+        if op == "decode_fp8":
+            k8, v8, kd, vd = quantise_e4m3(y, cfg, dev)
+            for _ in range(n):
+                abi.attn_sink_decode_fp8(y["q"], k8, v8, kd, vd, y["seqlens"], y["sinks"], cfg.W, cfg.scale, out)
+        elif op == "decode_paged":
+            kpool, vpool, table = page_cache(y, cfg, args.page, 0, dev)
+            del y["kcache"], y["vcache"]
+            for _ in range(n):
+                abi.attn_sink_decode_paged(y["q"], kpool, vpool, table, y["seqlens"], y["sinks"], cfg.W,
+                                           cfg.scale, out)
+        else:
+            for _ in range(n):
+                abi.attn_sink_decode(y["q"], y["kcache"], y["vcache"], y["seqlens"], y["sinks"],
+                                     cfg.W, cfg.scale, out)
+    torch.cuda.synchronize()
+    rc = abi.attn_sink_get_status()
+    print("ok" if rc == 0 else f"device status {rc}")
+    return 0 if rc == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -653,7 +879,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", choices=["fwd", "decode", "bwd", "decode_fp8", "decode_paged"],
+                    help="profiler driver: run --launches of one operation on --workload, no timing")
+    ap.add_argument("--workload", choices=sorted(_profile_workloads()), default="prefill")
+    ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--page", type=int, default=16, help="positions per page (--profile decode_paged)")
     args = ap.parse_args()
+    if args.profile:
+        sys.exit(run_profile(args))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -33,6 +33,12 @@
  *  - Device-side waits are bounded.  A wait that runs out records
  *    ATTN_ETIMEOUT in a device status word and the kernel returns early;
  *    attn_sink_get_status() reads and clears that word.
+ *  - Per device, the library looks up the device addresses of its own
+ *    device-side objects (the status word, the no-allocation scratch array)
+ *    once, and keeps its workspace pool and tensor-map cache for the life of
+ *    the process.  They belong to the device's primary context: do not use
+ *    the library on a device after cudaDeviceReset() (or any other teardown
+ *    of that primary context) in the same process.
  */
 #ifndef ATTNSINK_H
 #define ATTNSINK_H

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattnsink.so")
 SOURCES = ["api.cu", "fwd_tc.cu", "fwd_cudacore.cu", "decode.cu", "decode_noalloc.cu", "bwd.cu", "bwd_tc.cu"]
-HEADERS = ["ptx.cuh", "status.cuh", "kernels.h", "api_internal.h", "exp2_poly.h"]
+HEADERS = ["ptx.cuh", "status.cuh", "kernels.h", "api_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -32,7 +32,6 @@
 // lower edge or the end of the sequence.
 #include <math.h>
 
-#include "exp2_poly.h"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -47,9 +46,6 @@ constexpr uint32_t kBarEpilogue0 = 2;  // 2 + w: epilogue of warpgroup w
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-// Of every 8 columns of P, this many take the FMA-pipe polynomial for 2^x and
-// the rest the MUFU ex2 (the two pipes then finish at about the same time).
-constexpr int kPolyPerOctet = 0;
 // Instruction mix of the exponentiation pass (chosen by measurement).
 constexpr bool kPackedFma = true;   // f32x2 FMA for S*scale*log2e - m
 constexpr bool kPackedAdd = true;   // f32x2 adds for the row sum
@@ -191,32 +187,9 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for a packed pair on the FMA/ALU pipes (no MUFU).  Cody-Waite reduction
-// x = n + f, n = round(x) (via the 1.5*2^23 shifter), f in [-1/2, 1/2];
-// 2^f from the degree-3 fit of exp2_poly.h; 2^n added to the exponent field.
-// Inputs below -126 are clamped there (2^-126 ~ 1e-38 instead of 0).
-__device__ __forceinline__ void exp2_poly_x2(uint64_t x, float &y0, float &y1) {
-  const float kShift = 12582912.0f;                // 1.5 * 2^23
-  float x0, x1;
-  f2unpack(x, x0, x1);
-  x = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t = add2(x, f2pack(kShift, kShift));         // n in the low mantissa bits
-  const uint64_t nf = add2(t, f2pack(-kShift, -kShift));      // n as a float
-  const uint64_t f = add2(x, nf ^ 0x8000000080000000ull);     // x - n
-  uint64_t q = fma2(f, f2pack(kExp2C3, kExp2C3), f2pack(kExp2C2, kExp2C2));
-  q = fma2(q, f, f2pack(kExp2C1, kExp2C1));
-  q = fma2(q, f, f2pack(kExp2C0, kExp2C0));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(q0) + __float_as_uint(t0) * 8388608u);   // + n << 23
-  y1 = __uint_as_float(__float_as_uint(q1) + __float_as_uint(t1) * 8388608u);
-}
-
 // P = 2^(S*scale*log2e - m_use) for one row tile held in registers (sv),
 // written as bf16 over the first BN/2 columns at p_addr; returns the fp32 sum
-// of P, and with kMax also the tile's raw maximum in tmax.  Of every 8
-// columns kPolyPerOctet take the FMA-pipe polynomial for 2^x, the rest MUFU.
+// of P, and with kMax also the tile's raw maximum in tmax.
 template <int BN, bool kMax>
 __device__ __forceinline__ float exp_tile(const uint32_t (&sv)[BN / 32][32], uint32_t p_addr,
                                           float sl2, float m_use, uint32_t cls_none, float &tmax) {
@@ -243,13 +216,7 @@ __device__ __forceinline__ float exp_tile(const uint32_t (&sv)[BN / 32][32], uin
           z0 = fmaf(s0, sl2, -m_use);
           z1 = fmaf(s1, sl2, -m_use);
         }
-        float p0, p1;
-        if ((t & 3) < kPolyPerOctet / 2) {
-          exp2_poly_x2(f2pack(z0, z1), p0, p1);
-        } else {
-          p0 = ex2_approx(z0);
-          p1 = ex2_approx(z1);
-        }
+        const float p0 = ex2_approx(z0), p1 = ex2_approx(z1);
         if (kPackedAdd) {
           acc2[t & 1] = add2(acc2[t & 1], f2pack(p0, p1));
         } else {
