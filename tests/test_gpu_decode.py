@@ -107,10 +107,10 @@ def test_sink_minus_inf_and_dominant_sink():
         _check(o, ref, f"sinks {sk}")
 
 
-def test_decode_workload_sampled():
+def test_decode_workload_full():
     """B64 Hq32 Hkv4 D128, lengths ~ U[4096, 131072] (generated on the device):
-    every output finite and bounded; sampled sequences (the shortest, the
-    longest and a few others) against the oracle."""
+    every output of all 64 sequences against the fp64 oracle, one sequence at
+    a time (only its valid prefix of the cache comes to the host)."""
     cfg = inputs.DECODE
     y = inputs.make_decode(cfg, seed=0, device=DEV)
     out = torch.empty_like(y["q"])
@@ -121,10 +121,13 @@ def test_decode_workload_sampled():
     o = out.float().cpu().numpy()
     assert np.isfinite(o).all()
     sl = y["seqlens"].cpu().numpy()
-    pick = sorted({int(np.argmin(sl)), int(np.argmax(sl)), 0, 17, 63})
-    for b in pick:
+    sinks = y["sinks"].cpu().numpy()
+    worst = 0.0
+    for b in range(cfg.B):
         n = int(sl[b])
         ref = oracle.decode(inputs.bits(y["q"][b:b + 1]), inputs.bits(y["kcache"][b:b + 1, :n]),
                             inputs.bits(y["vcache"][b:b + 1, :n]), np.array([n], np.int32),
-                            y["sinks"].cpu().numpy(), cfg.W, cfg.scale)[0]
+                            sinks, cfg.W, cfg.scale)[0]
         _check(o[b:b + 1], ref, f"decode seq {b} (n={n})")
+        worst = max(worst, float(np.abs(o[b:b + 1] - ref).max()))
+    assert worst <= TOL_O

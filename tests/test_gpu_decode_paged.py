@@ -134,10 +134,11 @@ def test_paged_equals_contiguous_on_the_same_rows():
     assert err <= TOL_O, err
 
 
-def test_paged_decode_workload_sampled():
+def test_paged_decode_workload_full():
     """The decode workload (B64 Hq32 Hkv4 D128, lengths ~ U[4096, 131072])
     with its cache in 256-position pages at random pool positions: every
-    output finite; sampled sequences against the oracle."""
+    output finite, and all 64 sequences against the oracle (one at a time,
+    gathered from the pool by the block table on the device)."""
     cfg = inputs.DECODE
     P = 256
     y = inputs.make_decode(cfg, seed=0, device=DEV)
@@ -159,8 +160,7 @@ def test_paged_decode_workload_sampled():
     assert np.isfinite(o).all()
     sl = y["seqlens"].cpu().numpy()
     tab = table.cpu()
-    pick = sorted({int(np.argmin(sl)), int(np.argmax(sl)), 0, 17, 63})
-    for b in pick:
+    for b in range(B):
         n = int(sl[b])
         npg = (n + P - 1) // P
         rows = tab[b, :npg].to(DEV).long()

@@ -192,32 +192,14 @@ def test_stress_workload_full():
     np.testing.assert_allclose(lv[:, :8], 20.0, atol=TOL_LSE)
 
 
-def _sample_rows(B, L, Hq, n, rng):
-    """Rows spread over the sequence, plus the first, last and tile-edge rows."""
-    special = [0, 1, 127, 128, 129, L // 2, L - 129, L - 128, L - 1]
-    rows = []
-    for i in special:
-        for h in (0, Hq - 1):
-            rows.append((0, i, h))
-    rows += [(int(rng.integers(B)), int(rng.integers(L)), int(rng.integers(Hq))) for _ in range(n)]
-    return np.array(rows, dtype=np.int32)
-
-
-def test_long_causal_workload_sampled():
-    """B1 Hq32 Hkv8 L16384 D128 full causal: sampled rows against the oracle,
-    and every row against the CUDA-core implementation and the mass bound."""
+def test_long_causal_workload_full():
+    """B1 Hq32 Hkv8 L16384 D128 full causal (2.2 TFLOP): every output and LSE
+    against the fp64 oracle (about a minute and a half of oracle time on 16
+    host cores), plus the probability-mass bound |O| <= max|v|."""
     cfg = inputs.LONG_CAUSAL
     x = inputs.make_prefill(cfg, seed=0)
     o, lv = run_gpu(x, cfg.W, cfg.scale, "tc")
-    assert np.isfinite(o).all() and np.isfinite(lv).all()
-    rng = np.random.default_rng(0)
-    rows = _sample_rows(cfg.B, cfg.L, cfg.Hq, 600, rng)
-    ref_o, ref_l = oracle.fwd_rows(inputs.bits(x["q"]), inputs.bits(x["k"]), inputs.bits(x["v"]),
-                                   x["sinks"].numpy(), cfg.W, cfg.scale, rows)
-    got_o = o[rows[:, 0], rows[:, 1], rows[:, 2]]
-    got_l = lv[rows[:, 0], rows[:, 2], rows[:, 1]]
-    check(got_o, got_l, ref_o, ref_l, "long-causal sampled")
-    c, lc = run_gpu(x, cfg.W, cfg.scale, "cudacore")
-    assert float(np.abs(o - c).max()) <= TOL_O and float(np.abs(lv - lc).max()) <= TOL_LSE
+    ref_o, ref_l = oracle_fwd(x, cfg.W, cfg.scale)
+    check(o, lv, ref_o, ref_l, "long-causal")
     vmax = float(x["v"].float().abs().max())
     assert np.abs(o).max() <= vmax + TOL_O
