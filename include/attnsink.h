@@ -321,6 +321,27 @@ int attn_sink_decode_noalloc(const attn_tensor *q, const attn_tensor *kcache,
  */
 int attn_sink_get_status(void *stream);
 
+/*
+ * Diagnostics: failure injection for tests of the error paths.  Not needed in
+ * normal use (the pages have no counterpart to these).
+ *
+ * attn_sink_set_wait_limit_ns: the longest time any one device-side wait of
+ * the kernels launched from now on may take on the current device before it
+ * gives up, records ATTN_ETIMEOUT and lets its CTA return (0 restores the
+ * default of 1 s).  With a limit of a few nanoseconds, the first wait that is
+ * not satisfied at once gives up, so a call ends with ATTN_ETIMEOUT in the
+ * status word and an unspecified output; the library stays usable.  Waits
+ * that let a CTA's own copies land before it leaves keep the default limit.
+ * Synchronous (a host-to-device copy); the setting is per device and shared
+ * by every thread.
+ *
+ * attn_sink_fail_workspace_allocs: the next `count` workspace allocations
+ * (decode, paged, FP8 and backward calls, any thread) fail as if the pool had
+ * no memory: the call returns ATTN_ENOMEM and launches nothing.  0 cancels.
+ */
+int attn_sink_set_wait_limit_ns(uint64_t ns);
+int attn_sink_fail_workspace_allocs(int32_t count);
+
 /* Static description of an attn_status code. */
 const char *attn_sink_strerror(int code);
 

@@ -37,7 +37,7 @@ _DTYPES = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float32: ATTN_DTYPE_F32,
 EXPORTS = ("attn_sink_fwd", "attn_sink_fwd_max_logit", "attn_sink_fwd_varlen", "attn_sink_bwd", "attn_sink_fwd_cudacore", "attn_sink_decode",
            "attn_sink_decode_chunked", "attn_sink_decode_paged", "attn_sink_decode_fp8",
            "attn_sink_decode_noalloc",
-           "attn_sink_get_status",
+           "attn_sink_get_status", "attn_sink_set_wait_limit_ns", "attn_sink_fail_workspace_allocs",
            "attn_sink_strerror", "attn_sink_last_error")
 
 
@@ -88,6 +88,10 @@ def load() -> ctypes.CDLL:
         lib.attn_sink_decode_noalloc.restype = ctypes.c_int
         lib.attn_sink_get_status.argtypes = [V]
         lib.attn_sink_get_status.restype = ctypes.c_int
+        lib.attn_sink_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.attn_sink_set_wait_limit_ns.restype = ctypes.c_int
+        lib.attn_sink_fail_workspace_allocs.argtypes = [i32]
+        lib.attn_sink_fail_workspace_allocs.restype = ctypes.c_int
         lib.attn_sink_strerror.argtypes = [ctypes.c_int]
         lib.attn_sink_strerror.restype = ctypes.c_char_p
         lib.attn_sink_last_error.argtypes = []
@@ -256,6 +260,18 @@ def attn_sink_decode_noalloc(q, kcache, vcache, seqlens, sinks, window: int, sca
                                       _ref(ds[4]), int(window), float(scale), _ref(ds[5]),
                                       _stream(stream, q))
     _check(rc, "attn_sink_decode_noalloc")
+
+
+def attn_sink_set_wait_limit_ns(ns: int):
+    """C ``attn_sink_set_wait_limit_ns`` (diagnostics): limit of every device
+    wait on the current device, 0 = the default."""
+    _check(load().attn_sink_set_wait_limit_ns(int(ns)), "attn_sink_set_wait_limit_ns")
+
+
+def attn_sink_fail_workspace_allocs(count: int):
+    """C ``attn_sink_fail_workspace_allocs`` (diagnostics): the next ``count``
+    workspace allocations fail with ATTN_ENOMEM."""
+    _check(load().attn_sink_fail_workspace_allocs(int(count)), "attn_sink_fail_workspace_allocs")
 
 
 def attn_sink_get_status(stream=None) -> int:

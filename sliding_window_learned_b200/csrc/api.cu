@@ -9,6 +9,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/attnsink.h"
@@ -18,8 +19,10 @@
 namespace attnsink {
 
 // Device status word: [0] = first error code, [1] = location of the failing
-// wait.  Kernels receive its address; attn_sink_get_status reads and clears it.
-__device__ int g_status[2];
+// wait, [2..3] = the bounded waits' limit in ns (one 64-bit value; 0 = the
+// default).  Kernels receive its address; attn_sink_get_status reads and
+// clears [0..1]; attn_sink_set_wait_limit_ns sets [2..3].
+__device__ __align__(8) int g_status[4];
 
 namespace {
 thread_local char t_last_error[256] = "";
@@ -43,11 +46,22 @@ int fail_cuda(cudaError_t e, const char *what) {
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+// Injected workspace-allocation failures still to deliver
+// (attn_sink_fail_workspace_allocs).
+std::atomic<int> g_fail_allocs{0};
 int *g_status_ptr[kMaxDevices];
 cudaMemPool_t g_pool[kMaxDevices];
 bool g_pool_ready[kMaxDevices];
 
 }  // namespace
+
+// True (and one fewer to come) while injected allocation failures are pending.
+bool take_injected_alloc_failure() {
+  int n = g_fail_allocs.load();
+  while (n > 0)
+    if (g_fail_allocs.compare_exchange_weak(n, n - 1)) return true;
+  return false;
+}
 
 int current_device(int *dev) {
   const cudaError_t e = cudaGetDevice(dev);
@@ -762,6 +776,7 @@ int attn_sink_decode_chunked(const attn_tensor *q, const attn_tensor *kcache,
   const size_t bytes = decode_workspace_bytes(a);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void *ws = nullptr;
+  if (take_injected_alloc_failure()) return fail(ATTN_ENOMEM, "decode workspace allocation failed (injected)");
   cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, st);
   if (e != cudaSuccess) return fail_cuda(e, "decode workspace allocation");
   e = launch_decode(a, ws, st);
@@ -793,6 +808,7 @@ int attn_sink_decode_paged(const attn_tensor *q, const attn_tensor *kpages,
   const size_t bytes = decode_workspace_bytes(a);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void *ws = nullptr;
+  if (take_injected_alloc_failure()) return fail(ATTN_ENOMEM, "decode workspace allocation failed (injected)");
   cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, st);
   if (e != cudaSuccess) return fail_cuda(e, "decode workspace allocation");
   e = launch_decode(a, ws, st);
@@ -818,6 +834,7 @@ int attn_sink_decode_fp8(const attn_tensor *q, const attn_tensor *kcache, const 
   const size_t bytes = decode_workspace_bytes(a);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void *ws = nullptr;
+  if (take_injected_alloc_failure()) return fail(ATTN_ENOMEM, "decode workspace allocation failed (injected)");
   cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, st);
   if (e != cudaSuccess) return fail_cuda(e, "decode workspace allocation");
   e = launch_decode(a, ws, st);
@@ -843,12 +860,30 @@ int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
   cudaMemPool_t pool;
   if ((rc = workspace_pool(&pool))) return rc;
   void *ws = nullptr;
+  if (take_injected_alloc_failure()) return fail(ATTN_ENOMEM, "backward workspace allocation failed (injected)");
   cudaError_t e = cudaMallocFromPoolAsync(&ws, bwd_workspace_bytes(a), pool, st);
   if (e != cudaSuccess) return fail_cuda(e, "backward workspace allocation");
   e = launch_bwd(a, ws, st);
   const cudaError_t ef = cudaFreeAsync(ws, st);
   if (e != cudaSuccess) return fail_cuda(e, "attn_sink_bwd launch");
   if (ef != cudaSuccess) return fail_cuda(ef, "backward workspace release");
+  return ATTN_OK;
+}
+
+int attn_sink_set_wait_limit_ns(uint64_t ns) {
+  t_last_error[0] = '\0';
+  int *dptr;
+  int rc = status_ptr(&dptr);
+  if (rc) return rc;
+  const unsigned long long v = ns;
+  const cudaError_t e = cudaMemcpy(dptr + 2, &v, sizeof v, cudaMemcpyHostToDevice);
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e, "wait limit");
+}
+
+int attn_sink_fail_workspace_allocs(int32_t count) {
+  t_last_error[0] = '\0';
+  if (count < 0) return fail(ATTN_EINVAL, "count must be >= 0");
+  g_fail_allocs.store(count);
   return ATTN_OK;
 }
 

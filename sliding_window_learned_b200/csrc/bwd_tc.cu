@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *mma_done = dkv_free + 1;     // every product of the CTA finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-  const WaitCtx ctx{abort_flag, p.status};
+  const WaitCtx ctx{abort_flag, p.status, wait_limit_ns(p.status)};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -291,9 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++g;                                  // steps whose copies were issued
       }
     }
-    if (!ok && lane == 0) {
-      // Leaving early: let the copies already issued land before the CTA
-      // (and its shared memory) goes away.
+    if (lane == 0) {
+      // Before this warp leaves, the copies it issued have landed: the CTA
+      // (and its shared memory) must outlive them even when the other roles
+      // gave up early.  In a normal run they are long done.
       for (int k = max(0, kv_issued - kKVBuf); k < kv_issued; ++k)
         drain_wait(&kv_full[k % kKVBuf], static_cast<uint32_t>(k / kKVBuf) & 1u);
       for (int k = max(0, g - kStages); k < g; ++k)
@@ -519,7 +520,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < steps; ++s, ++g) {
         const int h = t.h0 + s / t.nq;
         const int i0 = (t.q_lo + s % t.nq) * kBQ;
-        if (!warp_wait(dq_full, static_cast<uint32_t>(g) & 1u, ctx, kWhereDq)) {
+        // the previous step's reduction has read the staging tile
+        if (rr == 0) tma_store_wait_read();
+        // The four warps' vote (the barrier that also publishes the read
+        // above): they go on, or leave, together, so the barrier below is
+        // met by all of them.
+        const bool got = warp_wait(dq_full, static_cast<uint32_t>(g) & 1u, ctx, kWhereDq);
+        if (!named_barrier_and(kBarDrain, 128, got)) {
           ok = false;
           break;
         }
@@ -530,9 +537,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(dq_empty);                        // the next dQ^T may overwrite it
-        // the previous step's reduction has read the staging tile
-        if (rr == 0) tma_store_wait_read();
-        named_barrier_sync(kBarDrain, 128);
         // dQ^T column -> dQ row-major tile: for each query the warp writes 32
         // consecutive channels
         if (rr < D) {                                 // (lanes past D hold padding)
@@ -549,7 +553,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_commit();
         }
         if (s == steps - 1) {
-          if (!warp_wait(dkv_full, static_cast<uint32_t>(ul) & 1u, ctx, kWhereDkv)) {
+          const bool kv_ok = warp_wait(dkv_full, static_cast<uint32_t>(ul) & 1u, ctx, kWhereDkv);
+          if (!named_barrier_and(kBarDrain, 128, kv_ok)) {
             ok = false;
             break;
           }

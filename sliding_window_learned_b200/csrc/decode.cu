@@ -43,10 +43,10 @@ namespace {
 
 constexpr int kTK = 64;               // keys per tile (bf16 cache)
 constexpr int kConsumerWarps = 4;     // each owns 16 keys of every tile (bf16 cache)
-constexpr uint32_t kBarMerge = 1;
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-enum : int { kWhereFull = 201, kWhereEmpty = 202 };
+enum : int { kWhereFull = 201, kWhereEmpty = 202, kWhereMerge = 203 };
 
 // Workspace layout (each section 256-byte aligned).
 struct WsLayout {
@@ -190,10 +190,11 @@ struct DCfg {
   static constexpr int kInfoOffset = kStages * kStageBytes + (kMergeInStage ? 0 : kMergeBytes);
   static_assert(!kMergeInStage || kCW * (NT / kMergePasses) * 8 * D * 4 <= kStageBytes,
                 "one merge pass fits a stage");
-  // stage descriptors, full/empty barriers, per-warp (max, sum) for the merge,
-  // the abort flag; plus 1 KB of slack for aligning the base to 1 KB
+  // stage descriptors, full/empty barriers, the consumers' merge barrier,
+  // per-warp (max, sum) for the merge, the abort flag; plus 1 KB of slack for
+  // aligning the base to 1 KB
   static constexpr int kInfoBytes =
-      (kStages * 32 + kStages * 16 + 2 * kCW * NT * 8 * 4 + 16 + 127) / 128 * 128;
+      (kStages * 32 + kStages * 16 + 8 + 2 * kCW * NT * 8 * 4 + 16 + 127) / 128 * 128;
   static constexpr int kSmemBytes = kInfoOffset + kInfoBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared-memory budget");
   static_assert(!kF8 || kInfoBytes <= 2048, "FP8 ring budget leaves room for the stage info");
@@ -224,6 +225,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, r);
 }
 
+// Before the producer leaves, the copies into the stages it armed have landed:
+// the CTA and its shared memory must outlive them, also when the consumers
+// gave up early.  `armed` stages were armed; only the last kStages of them
+// can still be in flight.  Each wait is bounded by the fixed limit, whatever
+// limit the other waits use.
+template <int kStages>
+__device__ __forceinline__ void drain_stages(uint64_t *full, int armed) {
+  for (int x = max(0, armed - kStages); x < armed; ++x) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&full[x % kStages], static_cast<uint32_t>(x / kStages) & 1u))
+      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
+}
+
 template <int D, int NT, bool kF8>
 __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -236,10 +251,11 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
   StageInfo *info = reinterpret_cast<StageInfo *>(smem + C::kInfoOffset);
   uint64_t *full = reinterpret_cast<uint64_t *>(info + C::kStages);
   uint64_t *empty = full + C::kStages;
-  float *merge_m = reinterpret_cast<float *>(empty + C::kStages);   // [4][NT*8]
+  uint64_t *merge_bar = empty + C::kStages;   // the consumer warps meet here around a merge
+  float *merge_m = reinterpret_cast<float *>(merge_bar + 1);   // [4][NT*8]
   float *merge_l = merge_m + C::kCW * NT * 8;               // [4][NT*8]
   int *abort_flag = reinterpret_cast<int *>(merge_l + C::kCW * NT * 8);
-  const WaitCtx ctx{abort_flag, p.status};
+  const WaitCtx ctx{abort_flag, p.status, wait_limit_ns(p.status)};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -248,6 +264,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], C::kCW);
     }
+    mbar_init(merge_bar, C::kCW * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -351,6 +368,8 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           mbar_arrive(&full[s]);
         }
       }
+      // (a failed acquire took a stage it never armed)
+      drain_stages<C::kStages>(full, ok ? slot : slot - 1);
     }
     // Pages smaller than a tile (several pages per tile): the whole warp
     // follows one control flow; lane 0 claims work, waits for free stages and
@@ -452,6 +471,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           mbar_arrive(&full[s]);
         }
       }
+      if (lane == 0) drain_stages<C::kStages>(full, ok ? slot : slot - 1);
     }
     __syncwarp();
     return;
@@ -478,6 +498,17 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
   uint32_t qf[D / 16][NT][2];     // B fragments of q^T, per k-step and head tile
   float o[D / 16][NT][4];         // O^T accumulators: [d tile][head tile][frag]
   float m_run[NT][2], l_run[NT][2];
+  // The consumer warps meet around each merge through an mbarrier (every
+  // consumer thread arrives, then waits for the phase, bounded): a warp that
+  // gave up on a wait leaves, and the others' next meeting then runs out
+  // instead of waiting for it forever.
+  uint32_t merge_phase = 0;
+  auto consumers_meet = [&]() -> bool {
+    mbar_arrive(merge_bar);
+    const bool met = warp_wait(merge_bar, merge_phase & 1u, ctx, kWhereMerge);
+    ++merge_phase;
+    return met;
+  };
   int slot = 0;
   while (true) {
     const int s = slot % C::kStages;
@@ -729,7 +760,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           l_run[nt][e] = l;
         }
       // previous merge fully read (FP8: and every warp done with this stage)
-      named_barrier_sync(kBarMerge, C::kCW * 32);
+      if (!consumers_meet()) return;
       if (g8 == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -747,7 +778,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       const int gsplit = p.base[si.b] + si.split;
 #pragma unroll
       for (int ps = 0; ps < C::kMergePasses; ++ps) {
-        if (ps > 0) named_barrier_sync(kBarMerge, C::kCW * 32);   // previous pass fully read
+        if (ps > 0 && !consumers_meet()) return;   // previous pass fully read
         float *mw = mbuf + warp * (kTP * 8 * D);  // [head of the pass][d]
 #pragma unroll
         for (int dm = 0; dm < D / 16; ++dm)
@@ -762,7 +793,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
             mw[hh * D + d1] = o[dm][nt][2];
             mw[(hh + 1) * D + d1] = o[dm][nt][3];
           }
-        named_barrier_sync(kBarMerge, C::kCW * 32);
+        if (!consumers_meet()) return;
         const int h0 = ps * kTP * 8;
         const int nh = min(p.G - h0, kTP * 8);
         for (int e = tid; e < nh * D; e += C::kCW * 32) {
@@ -787,7 +818,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
       if constexpr (C::kMergeInStage) {
         // every reader of the merge is done; its generic writes are ordered
         // before the next TMA write into the stage
-        named_barrier_sync(kBarMerge, C::kCW * 32);
+        if (!consumers_meet()) return;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);

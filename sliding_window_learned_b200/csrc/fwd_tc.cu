@@ -41,6 +41,7 @@ namespace {
 constexpr int kBM = 128;             // query rows per tile (= TMEM lanes)
 constexpr uint32_t kBarTmem = 1;     // named barrier ids (0 = __syncthreads);
 constexpr uint32_t kBarEpilogue0 = 2;  // 2 + w: epilogue of warpgroup w
+constexpr uint32_t kBarVote0 = 4;      // 4 + w: warpgroup w's vote on going on
 // Lazy rescaling: the running maximum (log2 units) only moves when a tile's
 // maximum exceeds it by more than this; until then exponents stay <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   uint64_t *mma_done = o_drained + NH;      // every MMA of the CTA finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-  const WaitCtx ctx{abort_flag, p.status};
+  const WaitCtx ctx{abort_flag, p.status, wait_limit_ns(p.status)};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -514,14 +515,15 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         }
       }
       (void)load;
-      if (!ok) {
-        // Leaving early: let the copies already issued land before the CTA
-        // (and its shared memory) goes away.
-        if (q_loaded > 0)
-          drain_wait(&q_full[(q_loaded - 1) & 1], static_cast<uint32_t>((q_loaded - 1) >> 1) & 1u);
-        for (int t = max(0, slot - C::kStages); t < slot; ++t)
-          drain_wait(&full[t % C::kStages], static_cast<uint32_t>(t / C::kStages) & 1u);
-      }
+      // Before this warp leaves, the copies it issued have landed: the CTA (and
+      // its shared memory) must outlive them even when the other roles gave
+      // up early.  Only the last two Q loads and the last kStages K/V tiles
+      // can still be in flight (every earlier one was waited for before its
+      // buffer was reused).  In a normal run they are long done.
+      for (int uq = max(0, q_loaded - 2); uq < q_loaded; ++uq)
+        drain_wait(&q_full[uq & 1], static_cast<uint32_t>(uq >> 1) & 1u);
+      for (int t = max(0, slot - C::kStages); t < slot; ++t)
+        drain_wait(&full[t % C::kStages], static_cast<uint32_t>(t / C::kStages) & 1u);
     }
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
@@ -677,7 +679,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       float m_run = -INFINITY;                       // running max, log2 units
       float row_max = -INFINITY;                     // exact row maximum, log2 units
       float l_run = 0.f;                             // running denominator
-      for (int j = 0; j < t.n_tiles; ++j) {
+      for (int j = 0; ok && j < t.n_tiles; ++j) {
         const int g = jg + j;
         const uint32_t s_col = C::kSCol(w, g % C::kSBuf);
         if (!warp_wait(&s_full[2 * w + g % C::kSBuf], static_cast<uint32_t>(g / C::kSBuf) & 1u,
@@ -722,7 +724,12 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         }
       }
       jg += t.n_tiles;
-      if (ok) ok = warp_wait(&o_full[w], static_cast<uint32_t>(ul) & 1u, ctx, kWhereO);
+      bool w_ok = false;
+      if (ok) w_ok = warp_wait(&o_full[w], static_cast<uint32_t>(ul) & 1u, ctx, kWhereO);
+      // Every warp of the warpgroup reaches this vote once per unit (a warp
+      // whose bounded wait ran out leaves its tile loop early and comes here),
+      // so the epilogue's barrier below is met by all four warps or by none.
+      ok = named_barrier_and(kBarVote0 + w, 128, w_ok);
       if (!ok) break;
       tc_fence_after();
       // ---- sink epilogue (page "cf-1.com/news/6055759", fix 2) ----

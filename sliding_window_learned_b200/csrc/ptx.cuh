@@ -81,17 +81,21 @@ constexpr uint32_t kWaitSleepNs = 50000;
 
 // Bounded wait for the phase with the given parity.  The thread sleeps in the
 // barrier (woken when the phase completes); each time it wakes without the
-// phase it checks the CTA abort flag and the elapsed time.  On timeout it
+// phase it checks the CTA abort flag and the elapsed time against the
+// launch's limit (1 s unless set otherwise in the status word).  On timeout it
 // records ATTN_ETIMEOUT (with `where` as the location code), raises the abort
 // flag so that the rest of the CTA stops waiting too, and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtx &ctx,
                                           int where) {
-  if (mbar_try_wait(bar, parity)) return true;
+  // (a first probe that may block briefly in hardware; skipped under a
+  // diagnostic limit shorter than one sleep, so that short waits run out too)
+  if (ctx.limit >= kWaitSleepNs && mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = ctx.limit < kWaitSleepNs ? static_cast<uint32_t>(ctx.limit) : kWaitSleepNs;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (*ctx.abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > ctx.limit) {
       report_timeout(ctx.status, where);
       *ctx.abort = 1;
       return false;
@@ -106,6 +110,23 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also reduces a predicate over its participants: true
+// for every participant iff `pred` was true for all of them.
+// Used after bounded waits, so that the threads that meet at later barriers
+// all take the same way out when one of them gave up.
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ----------------------------------------------------------------------- TMA

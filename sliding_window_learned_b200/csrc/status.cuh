@@ -13,11 +13,21 @@ constexpr int kStatusTimeout = -5;
 
 // Per-CTA context for bounded waits: a shared abort flag (so one timed-out
 // wait stops the whole CTA promptly) and the global status word
-// ([0] = code, [1] = location of the first failing wait).
+// ([0] = code, [1] = location of the first failing wait, [2..3] = the wait
+// limit in ns as one 64-bit value, 0 = kWaitLimitNs).
 struct WaitCtx {
   volatile int *abort;
   int *status;
+  uint64_t limit;   // this launch's wait limit in ns (read once, at the start)
 };
+
+// The limit a bounded wait uses: the one set in the status word, else the
+// default.  (Waits that drain in-flight copies on the way out keep the
+// default, so that a short limit never lets a CTA leave with copies landing.)
+__device__ __forceinline__ uint64_t wait_limit_ns(const int *status) {
+  const unsigned long long v = *reinterpret_cast<const volatile unsigned long long *>(status + 2);
+  return v == 0 ? kWaitLimitNs : static_cast<uint64_t>(v);
+}
 
 __device__ __forceinline__ void report_timeout(int *status, int where) {
   if (atomicCAS(status, 0, kStatusTimeout) == 0) atomicExch(status + 1, where);
