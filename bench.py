@@ -12,7 +12,8 @@ GB/s of algorithmic bytes) is reported beside it, and after the timed steps
 the same decode over a paged copy of its cache (256-position pages at random
 pool positions, attn_sink_decode_paged) is timed as `decode_paged`, the decode
 over the cache quantised to e4m3 (attn_sink_decode_fp8) as `decode_fp8`, the
-forward over a seeded mix of 24 packed sequences (attn_sink_fwd_varlen) as
+bf16 and e4m3 caches side by side on two more decode shapes (16 query heads per
+kv head; head dim 256) as `decode_shapes`, the forward over a seeded mix of 24 packed sequences (attn_sink_fwd_varlen) as
 `fwd_varlen`, and the backward pass on the prefill workload (attn_sink_bwd) as
 `bwd`.  `workloads` times attn_sink_fwd on each prefill workload on its own
 (tiny, prefill, long causal, sink stress), each with its own clock record.
@@ -450,6 +451,37 @@ def run_ours(args, rank, world, local_rank):
     dbytes8 = (dbytes - 2 * dcfg.B * dcfg.Hq * dcfg.D * 2) // 2 + 2 * dcfg.B * dcfg.Hq * dcfg.D * 2
     del k8, v8
 
+    # ---- two more decode shapes, bf16 and FP8 caches side by side ----
+    shape_times = []
+    shape_bytes = []
+    for si, scfg in enumerate((inputs.DECODE_G16, inputs.DECODE_D256)):
+        ys = inputs.make_decode(scfg, seed=2000 + 10 * si + rank, device=dev)
+        sout = torch.empty_like(ys["q"])
+        s8 = quantise_e4m3(ys, scfg, dev)
+        sl = ys["seqlens"].cpu().numpy().astype(np.int64)
+        qo_bytes = 2 * scfg.B * scfg.Hq * scfg.D * 2
+        b16 = int(sl.sum()) * scfg.Hkv * scfg.D * 2 * 2 + qo_bytes
+        shape_bytes.append((scfg.name, b16, (b16 - qo_bytes) // 2 + qo_bytes))
+        calls = (lambda: swl.attn_sink_decode(ys["q"], ys["kcache"], ys["vcache"], ys["seqlens"], ys["sinks"],
+                                              scfg.W, scfg.scale, sout, stream),
+                 lambda: swl.attn_sink_decode_fp8(ys["q"], s8[0], s8[1], s8[2], s8[3], ys["seqlens"], ys["sinks"],
+                                                  scfg.W, scfg.scale, sout, stream))
+        for call in calls:
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(Kp):
+                call()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if swl.attn_sink_get_status() != 0:
+                raise RuntimeError(f"device status error in the {scfg.name} decode")
+            shape_times.append(e0.elapsed_time(e1) / 1e3)
+        del ys, sout, s8
+        torch.cuda.empty_cache()
+    shape_times = max_over_ranks(shape_times, world, dev)
+
     # ---- the forward over packed variable-length sequences: a seeded mix of
     # 24 sequences of U[1, 4096] tokens at the prefill workload's heads ----
     vl_rng = np.random.default_rng(1000 + rank)
@@ -635,6 +667,15 @@ def run_ours(args, rank, world, local_rank):
                            "sliding_window_learned_b200/csrc/ptx.cuh"]),
                        "what": "attn_sink_decode_fp8 on the decode workload, cache quantised to e4m3 per "
                                "kv head (bytes counted at one per element)"},
+        "decode_shapes": {nm: {
+            "bf16": {"value": round(aggregate_rate(Kp * b16, world, shape_times[2 * i]) / 1e9, 2), "unit": "GB/s",
+                     "ms_per_call": round(shape_times[2 * i] / Kp * 1e3, 4),
+                     "frac": round(b16 / (shape_times[2 * i] / Kp) / 1e9 / hbm_peak, 4)},
+            "fp8": {"value": round(aggregate_rate(Kp * b8, world, shape_times[2 * i + 1]) / 1e9, 2), "unit": "GB/s",
+                    "ms_per_call": round(shape_times[2 * i + 1] / Kp * 1e3, 4),
+                    "frac": round(b8 / (shape_times[2 * i + 1] / Kp) / 1e9 / hbm_peak, 4)},
+            "fp8_rate_over_bf16": round((b8 / shape_times[2 * i + 1]) / (b16 / shape_times[2 * i]), 4)}
+            for i, (nm, b16, b8) in enumerate(shape_bytes)},
         "fwd_varlen": {"value": round(aggregate_rate(Kv * vl_flops, world, t_varlen) / 1e12, 3), "unit": "TFLOP/s",
                        "ms_per_call": round(t_varlen / Kv * 1e3, 5),
                        "frac": round(vl_flops / (t_varlen / Kv) / 1e12 / bf16_peak, 4),
@@ -807,6 +848,11 @@ def _profile_workloads():
         # same length distribution as the decode workload, 8 sequences (~1 GB of cache)
         "decode-small": inputs.Decode("decode-small B8 Hq32 Hkv4 D128 n~U[4096,131072]", 8, 32, 4,
                                       128, 131072, 4096, 131072, 131072),
+        # the two extra decode shapes at 8 and 4 sequences (~1 GB of cache each)
+        "decode-g16-small": inputs.Decode("decode-g16-small B8 Hq64 Hkv4 D128 n~U[4096,131072]", 8, 64, 4,
+                                          128, 131072, 4096, 131072, 131072),
+        "decode-d256-small": inputs.Decode("decode-d256-small B4 Hq32 Hkv4 D256 n~U[4096,131072]", 4, 32, 4,
+                                           256, 131072, 4096, 131072, 131072),
     }
 
 

@@ -13,11 +13,12 @@
 //            table names: one box per tile, or for pages of 16 or 32
 //            positions one box per page holding every channel chunk, through
 //            a 5-D view of the pool);
-//            four consumer warps each take 16 keys of every tile and run
+//            the consumer warps (four for a 16-bit cache; twelve, or eight at
+//            D = 256, for an FP8 cache) each take 16 keys of every tile and run
 //            S^T = K q^T and O^T += V^T P^T on the warp-level tensor cores
 //            (the Hq/Hkv grouped query heads are the N = 8 dimension), with an
 //            online softmax per head and NO sink.  At the end of an item the
-//            four warps' (max, sum, O) are merged and one normalised partial
+//            warps' (max, sum, O) are merged and one normalised partial
 //            (O_s, LSE_s) per query head is written.
 //   combine  one warp per (sequence, query head): merges exactly the splits
 //            that exist, in split order, and adds the sink once.
@@ -174,7 +175,14 @@ struct StageInfo {
 // which is released after it; the ring takes all the rest of shared memory.
 template <int D, int NT, bool kF8>
 struct DCfg {
-  static constexpr int kCW = (kF8 && D == 128) ? (NT == 1 ? 12 : 8) : kConsumerWarps;   // consumer warps
+  // consumer warps: FP8 caches take more warps per scheduler to hide the
+  // conversion latency (D = 256: eight, as many as three 64 KB stages and the
+  // merge in one stage allow)
+  static constexpr int kCW = kF8 ? (D == 128 ? 12 : 8) : kConsumerWarps;
+  // FP8 cache, two head tiles: each consumer warp keeps its q fragments in a
+  // private slice of shared memory instead of 32 registers, so that twelve
+  // consumer warps (four warps per scheduler, 128 registers each) fit
+  static constexpr bool kQInSmem = kF8 && NT == 2;
   static constexpr int kTK = 16 * kCW;                    // keys per tile
   static constexpr int kThreads = (kCW + 1) * 32;         // + the producer warp
   static constexpr bool kMergeInStage = kF8;
@@ -184,10 +192,12 @@ struct DCfg {
   static constexpr int kTileBytes = kTK * D * (kF8 ? 1 : 2);   // one K (or V) tile as stored
   static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
   static constexpr int kMergeBytes = kCW * NT * 8 * D * 4;
-  static constexpr int kRingBudget = kF8 ? 232448 - 1024 - 2048 : 196608 - kMergeBytes;
+  static constexpr int kQBytes = kQInSmem ? kCW * (D / 16) * NT * 32 * 8 : 0;   // [warp][kk][nt][lane] uint2
+  static constexpr int kRingBudget = kF8 ? 232448 - 1024 - 2048 - kQBytes : 196608 - kMergeBytes;
   static constexpr int kStages = (kRingBudget / kStageBytes) > 12 ? 12 : (kRingBudget / kStageBytes);
   static constexpr int kMergeOffset = kStages * kStageBytes;   // (16-bit cache only)
-  static constexpr int kInfoOffset = kStages * kStageBytes + (kMergeInStage ? 0 : kMergeBytes);
+  static constexpr int kQOffset = kStages * kStageBytes;       // (kQInSmem only)
+  static constexpr int kInfoOffset = kStages * kStageBytes + (kMergeInStage ? 0 : kMergeBytes) + kQBytes;
   static_assert(!kMergeInStage || kCW * (NT / kMergePasses) * 8 * D * 4 <= kStageBytes,
                 "one merge pass fits a stage");
   // stage descriptors, full/empty barriers, the consumers' merge barrier,
@@ -495,7 +505,10 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
   const uint32_t zrow_off = row_off(key_w + (lane & 15));        // V rows zeroed by lanes l, l + 16
   float sl2 = p.scale_log2;       // (FP8: times the item's key descale)
   float vdesc = 1.f;              // (FP8: the item's value descale)
-  uint32_t qf[D / 16][NT][2];     // B fragments of q^T, per k-step and head tile
+  // B fragments of q^T, per k-step and head tile (kQInSmem: the item's copy
+  // lives in this warp's slice of shared memory between tiles)
+  uint32_t qf[C::kQInSmem ? 1 : D / 16][NT][2];
+  uint2 *qsm = reinterpret_cast<uint2 *>(smem + C::kQOffset) + warp * (D / 16) * NT * 32 + lane;
   float o[D / 16][NT][4];         // O^T accumulators: [d tile][head tile][frag]
   float m_run[NT][2], l_run[NT][2];
   // The consumer warps meet around each merge through an mbarrier (every
@@ -520,6 +533,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     const uint32_t vbase = kbase + C::kTileBytes;
     if (si.flags & 1) {
       // first tile of a work item: load this kv head's grouped queries
+      uint32_t qx[D / 16][NT][2];
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
 #pragma unroll
@@ -534,8 +548,8 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
             x0 = *reinterpret_cast<const uint32_t *>(qr);
             x1 = *reinterpret_cast<const uint32_t *>(qr + (kF8 ? 2 : 8));
           }
-          qf[kk][nt][0] = x0;
-          qf[kk][nt][1] = x1;
+          qx[kk][nt][0] = x0;
+          qx[kk][nt][1] = x1;
         }
 #pragma unroll
       for (int dm = 0; dm < D / 16; ++dm)
@@ -559,7 +573,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int f = 0; f < 2; ++f) {
-              const uint32_t x = qf[kk][nt][f];
+              const uint32_t x = qx[kk][nt][f];
               mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(x << 16)), fabsf(__uint_as_float(x & 0xFFFF0000u))));
             }
 #pragma unroll
@@ -572,9 +586,24 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int f = 0; f < 2; ++f) qf[kk][nt][f] = bf16x2_to_f16x2_scaled(qf[kk][nt][f], qs);
+            for (int f = 0; f < 2; ++f) qx[kk][nt][f] = bf16x2_to_f16x2_scaled(qx[kk][nt][f], qs);
         sl2 = p.scale_log2 * p.k_descale[si.hk] * ldexpf(1.f, -e);
         vdesc = p.v_descale[si.hk];
+      }
+      if constexpr (C::kQInSmem) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) qsm[(kk * NT + nt) * 32] = make_uint2(qx[kk][nt][0], qx[kk][nt][1]);
+        __syncwarp();
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            qf[kk][nt][0] = qx[kk][nt][0];
+            qf[kk][nt][1] = qx[kk][nt][1];
+          }
       }
     }
     // Keys past the end of the split, and (paged cache) keys before the
@@ -619,8 +648,16 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
           const int kk = c8 * 8 + 2 * up;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            mma_f16_16816(sacc[nt], k0.x, k1.x, k0.y, k1.y, qf[kk][nt][0], qf[kk][nt][1]);
-            mma_f16_16816(sacc[nt], k2.x, k3.x, k2.y, k3.y, qf[kk + 1][nt][0], qf[kk + 1][nt][1]);
+            uint2 qa, qb;
+            if constexpr (C::kQInSmem) {
+              qa = qsm[(kk * NT + nt) * 32];
+              qb = qsm[((kk + 1) * NT + nt) * 32];
+            } else {
+              qa = make_uint2(qf[kk][nt][0], qf[kk][nt][1]);
+              qb = make_uint2(qf[kk + 1][nt][0], qf[kk + 1][nt][1]);
+            }
+            mma_f16_16816(sacc[nt], k0.x, k1.x, k0.y, k1.y, qa.x, qa.y);
+            mma_f16_16816(sacc[nt], k2.x, k3.x, k2.y, k3.y, qb.x, qb.y);
           }
         }
     } else {
@@ -749,7 +786,7 @@ __global__ void __launch_bounds__(DCfg<D, NT, kF8>::kThreads, 1)
     }
 
     if (si.flags & 2) {
-      // ---- merge the four warps' partial states and write (O_s, LSE_s) ----
+      // ---- merge the consumer warps' partial states and write (O_s, LSE_s) ----
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll

@@ -67,6 +67,12 @@ LONG_CAUSAL = Prefill("long causal B1 Hq32 Hkv8 L16384 D128 W=L", 1, 16384, 32, 
                       16384, ("normal", 0.0, 2.0))
 DECODE = Decode("split-KV decode B64 Hq32 Hkv4 D128 n~U[4096,131072]", 64, 32, 4, 128,
                 131072, 4096, 131072, 131072)
+# Two more decode shapes, for the bf16 and FP8 caches side by side: 16 query
+# heads per kv head (two 8-head tiles per kv head), and head dim 256.
+DECODE_G16 = Decode("decode G16 B64 Hq64 Hkv4 D128 n~U[4096,131072]", 64, 64, 4, 128,
+                    131072, 4096, 131072, 131072)
+DECODE_D256 = Decode("decode D256 B32 Hq32 Hkv4 D256 n~U[4096,131072]", 32, 32, 4, 256,
+                     131072, 4096, 131072, 131072)
 # Content logits near -150: q = z1 + c, k = z2 - c with c = sqrt(150 / (D*scale)).
 STRESS = Prefill("sink stress B1 Hq16 Hkv2 L8192 D256 W513", 1, 8192, 16, 2, 256, 513,
                  ("split", 20.0, -50.0), qk_offset=math.sqrt(150.0 / (256 * (1 / 16))))

@@ -72,6 +72,10 @@ CASES = [  # B, Smax, Hq, Hkv, D, W, seqlens
     (2, 700, 16, 1, 128, 256, [700, 300]),
     (3, 333, 8, 2, 256, 1 << 30, [333, 100, 0]),
     (2, 1024, 6, 2, 256, 513, [1024, 600]),
+    # many splits and 192-key tiles of the 16-heads-per-kv-head kernel (q
+    # fragments in shared memory), and of the eight-warp D = 256 kernel
+    (2, 20000, 32, 2, 128, 1 << 30, [20000, 12345]),
+    (2, 20000, 16, 2, 256, 4096, [20000, 7777]),
 ]
 
 
