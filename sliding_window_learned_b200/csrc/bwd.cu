@@ -28,11 +28,12 @@
 namespace attnsink {
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ rows
 // Dsum[b, h, i] = dO . O for every row, and dsink[h] -= exp(sink - LSE) * Dsum
-// (one atomic per block).  A block takes 64 rows of one (batch, head); each
+// (one atomic per block).  The block also zeroes its rows of the fp32 dQ
+// accumulator, and (blocks of the first Hkv heads) those of dK and dV, which
+// the main pass then adds into.  A block takes 64 rows of one (batch, head); each
 // warp takes 8 of them with every load issued before the first sum, each lane
 // D/32 consecutive channels (vector loads when the rows are aligned).
 template <int E, bool kVec, typename T>
@@ -59,13 +60,29 @@ __device__ __forceinline__ void load_row(const T *p, float (&v)[E]) {
 template <typename OT, int D, bool kVec>
 __global__ void __launch_bounds__(256) bwd_rows_kernel(const OT *o, const __nv_bfloat16 *dout,
                                                        const float *lse, const float *sinks, float *dsum,
-                                                       float *dsink, int L, int Hq, int64_t o_sb,
+                                                       float *dsink, float *dq_acc, float *dk_acc, float *dv_acc,
+                                                       int L, int Hq, int Hkv, int64_t o_sb,
                                                        int64_t o_sl, int64_t o_sh, int64_t d_sb, int64_t d_sl,
                                                        int64_t d_sh, int64_t lse_sb, int64_t lse_sh) {
   constexpr int E = D / 32;
   const int h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i0 = blockIdx.x * 64 + warp;             // rows i0, i0 + 8, ..., i0 + 56
+  {
+    // zero this block's accumulator rows (16-byte stores, a row's D floats
+    // by consecutive threads)
+    const int nrow = min(64, L - static_cast<int>(blockIdx.x) * 64);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t row0 = static_cast<int64_t>(b) * L + static_cast<int64_t>(blockIdx.x) * 64;
+    for (int e = threadIdx.x; e < nrow * (D / 4); e += 256) {
+      const int r = e / (D / 4), c = (e - r * (D / 4)) * 4;
+      *reinterpret_cast<float4 *>(dq_acc + ((row0 + r) * Hq + h) * D + c) = z;
+      if (h < Hkv) {
+        *reinterpret_cast<float4 *>(dk_acc + ((row0 + r) * Hkv + h) * D + c) = z;
+        *reinterpret_cast<float4 *>(dv_acc + ((row0 + r) * Hkv + h) * D + c) = z;
+      }
+    }
+  }
   float acc[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -156,10 +173,9 @@ cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
   const size_t kv_bytes = sizeof(float) * static_cast<size_t>(a.B) * a.L * a.Hkv * a.D;
   float *dk_acc = reinterpret_cast<float *>(ws + align256(acc_bytes) + align256(ds_bytes));
   float *dv_acc = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(dk_acc) + align256(kv_bytes));
-  cudaError_t e = cudaMemsetAsync(dq_acc, 0, acc_bytes, stream);
+  // (the row kernel zeroes the dQ, dK and dV accumulators)
+  cudaError_t e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.Hq, stream);
   if (e != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(dk_acc, 0, align256(kv_bytes) + kv_bytes, stream)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(a.dsink, 0, sizeof(float) * a.Hq, stream)) != cudaSuccess) return e;
   dim3 rg((a.L + 63) / 64, a.Hq, a.B);
   // vector loads of O need its rows aligned to the per-lane chunk (bf16 rows
   // are: their strides and base are 16-byte multiples)
@@ -171,7 +187,7 @@ cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
     using OT = decltype(ot);
     bwd_rows_kernel<OT, decltype(dconst)::value, decltype(vec)::value><<<rg, 256, 0, stream>>>(
         static_cast<const OT *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.sinks, dsum, a.dsink,
-        a.L, a.Hq, a.o_s[0], a.o_s[1], a.o_s[2], a.do_s[0], a.do_s[1], a.do_s[2], a.lse_s[0], a.lse_s[1]);
+        dq_acc, dk_acc, dv_acc, a.L, a.Hq, a.Hkv, a.o_s[0], a.o_s[1], a.o_s[2], a.do_s[0], a.do_s[1], a.do_s[2], a.lse_s[0], a.lse_s[1]);
   };
   using D64 = std::integral_constant<int, 64>;
   using D128 = std::integral_constant<int, 128>;
