@@ -112,6 +112,14 @@ CASES = [
     (1, 513, 4, 2, 256, 513, ("split", 20.0, -50.0)),
     (2, 333, 8, 8, 256, 1000, ("normal", 0, 2)),
     (1, 64, 2, 1, 256, 1, ("uniform", -4, 8)),
+    # one query head per kv head, or an odd group: the one-head kernel, over
+    # several query tiles with ragged tails
+    (2, 1000, 4, 4, 128, 513, ("uniform", -4, 8)),
+    (1, 512, 3, 1, 128, 1, ("uniform", -4, 8)),
+    (1, 768, 6, 2, 128, 129, ("normal", 0, 2)),
+    (2, 256, 2, 2, 64, 200, ("uniform", -4, 8)),
+    (1, 900, 4, 4, 64, 300, ("const", 30.0)),
+    (1, 640, 4, 4, 128, 513, ("uniform", -4, 8)),
 ]
 
 

@@ -54,6 +54,7 @@ CASES = [  # B, L, Hq, Hkv, D, W
     (2, 517, 4, 4, 64, 1 << 30),
     (1, 400, 4, 2, 256, 129),
     (1, 333, 3, 1, 128, 50),
+    (2, 1024, 4, 4, 128, 513),
 ]
 
 
