@@ -13,20 +13,22 @@
 // written for sm_100a directly.
 //
 // One CTA computes one 128-row query tile for NH query heads of the same
-// kv-head group (NH = 2 when the group size is even).  Those heads read the
-// same K/V tiles under the same mask, so every K/V tile brought from L2 feeds
-// NH x 128 query rows.  Warps:
+// kv-head group.  The dispatched form is NH = 1: one head per CTA, 64-key
+// tiles, two S buffers (S_{j+1} is computed while tile j is exponentiated),
+// 256 TMEM columns, so two CTAs share each SM and their MMA streams and
+// exponentials interleave.  (NH = 2, two heads of a group sharing each
+// 128-key K/V tile in one CTA, measured slower on every workload.)  Warps:
 //   0 .. 4*NH-1  softmax / correction / epilogue: warpgroup w owns head slot
 //                w, one thread per query row (TMEM lane)
-//   4*NH         TMA producer: Q (NH tiles) once, then K_0, V_0, K_1, V_1, ...
+//   4*NH         TMA producer: Q (NH tiles) once, then K_0, K_1, then V_j,
+//                K_{j+2} per tile (one S buffer: K_0, then V_j, K_{j+1})
 //                into a ring of shared-memory stages
-//   4*NH+1       TMEM allocator and MMA issuer, in the order
-//                S^0_0, S^1_0, then per key tile j:
-//                  PV^0_j, S^0_{j+1}, PV^1_j, S^1_{j+1}
-//                so that while one warpgroup exponentiates, the tensor cores
-//                work for the other (ping-pong).
-// TMEM (columns): S^w at w*BN (P^w written as bf16 over its first BN/2
-// columns), O^w at NH*BN + w*D.
+//   4*NH+1       TMEM allocator and MMA issuer: per key tile j and head w,
+//                PV^w_j then the S^w it frees a buffer for, so that the
+//                tensor cores compute one tile while the softmax works on
+//                another.
+// TMEM (columns): S^w buffer b at (kSBuf*w + b)*BN (P^w written as bf16 over
+// its first BN/2 columns), O^w after all S buffers.
 // Only the K tiles that meet the window [m0-W+1, m0+127] are visited; the
 // mask is applied on the tiles that cross the causal diagonal, the window's
 // lower edge or the end of the sequence.
@@ -898,21 +900,21 @@ cudaError_t launch_max_logit_init(float *ml, int64_t sb, int B, int Hq, cudaStre
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream) {
-  // Two query heads per CTA when they share a kv head (even group size) and
-  // their S and O fit TMEM together; otherwise one.
-  const bool pair = (a.Hq / a.Hkv) % 2 == 0;
+  // One query head per CTA, 64-key tiles with two S buffers, two CTAs per SM,
+  // for every group size.  (The kernel also takes two query heads of a kv
+  // group per CTA, NH = 2, sharing each K/V tile; measured on B200 that was
+  // slower on every workload: W = 513 534 against 587 TFLOP/s, full causal
+  // 967 against 1051, packed sequences 7-11 % slower.)
   const bool packed = a.cu_seqlens != nullptr;
   const bool ml = a.max_logit != nullptr;   // (batched inputs only)
   if (packed && ml) return cudaErrorInvalidValue;
   switch (a.D) {
     case 64:
-      if (packed) return pair ? launch<64, 128, 2, true>(a, stream) : launch<64, 64, 1, true>(a, stream);
-      if (ml) return pair ? launch<64, 128, 2, false, true>(a, stream) : launch<64, 64, 1, false, true>(a, stream);
-      return pair ? launch<64, 128, 2, false>(a, stream) : launch<64, 64, 1, false>(a, stream);
+      if (packed) return launch<64, 64, 1, true>(a, stream);
+      return ml ? launch<64, 64, 1, false, true>(a, stream) : launch<64, 64, 1, false>(a, stream);
     case 128:
-      if (packed) return pair ? launch<128, 128, 2, true>(a, stream) : launch<128, 64, 1, true>(a, stream);
-      if (ml) return pair ? launch<128, 128, 2, false, true>(a, stream) : launch<128, 64, 1, false, true>(a, stream);
-      return pair ? launch<128, 128, 2, false>(a, stream) : launch<128, 64, 1, false>(a, stream);
+      if (packed) return launch<128, 64, 1, true>(a, stream);
+      return ml ? launch<128, 64, 1, false, true>(a, stream) : launch<128, 64, 1, false>(a, stream);
     case 256:
       if (packed) return launch<256, 64, 1, true>(a, stream);
       return ml ? launch<256, 64, 1, false, true>(a, stream) : launch<256, 64, 1, false>(a, stream);

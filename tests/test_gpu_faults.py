@@ -53,8 +53,8 @@ def _timed_out(call):
         swl.attn_sink_set_wait_limit_ns(0)
 
 
-# (B, L, Hq, Hkv, D, W): the two-head tensor-core kernel, the one-head one,
-# and head dim 256
+# (B, L, Hq, Hkv, D, W): head dims 64, 128 and 256 of the tensor-core kernel,
+# with groups of 2 and 3 query heads and two kv heads
 FWD_CASES = [(1, 128, 2, 1, 64, 64), (1, 200, 3, 1, 128, 100), (1, 130, 2, 2, 256, 64)]
 
 
