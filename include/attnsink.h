@@ -317,7 +317,9 @@ int attn_sink_decode_noalloc(const attn_tensor *q, const attn_tensor *kcache,
 /*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, ATTN_ETIMEOUT (a bounded wait ran out), or
- * ATTN_ECUDA if the synchronisation itself failed.
+ * ATTN_ECUDA if the synchronisation itself failed or a kernel found its launch
+ * unusable (its dynamic shared memory not at the declared 1024-byte
+ * alignment; it then returns before doing any work).
  */
 int attn_sink_get_status(void *stream);
 

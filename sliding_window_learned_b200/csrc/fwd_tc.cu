@@ -56,7 +56,7 @@ constexpr bool kFusedMax = true;    // tile maximum in the same pass (else: sum 
 
 // wait-location codes reported with ATTN_ETIMEOUT
 enum : int { kWhereQ = 101, kWhereFull = 102, kWhereEmpty = 103, kWhereS = 104, kWhereP = 105,
-             kWhereO = 106 };
+             kWhereO = 106, kWhereAlign = 107 };
 
 template <int D, int BN, int NH>
 struct Cfg {
@@ -78,7 +78,7 @@ struct Cfg {
   static constexpr uint32_t kTmemThreads = 32u * __builtin_popcount(kTmemWarpMask);
 
   static constexpr int kChunks = D / 64;          // 64-channel (128-byte) column chunks
-  static constexpr int kBarBytes = 512;           // mbarriers, TMEM base, abort flag
+  static constexpr int kBarBytes = 256;           // mbarriers, TMEM base, abort flag
   static constexpr int kQTileBytes = kBM * D * 2;
   static constexpr int kQBufBytes = NH * kQTileBytes;   // one unit's Q tiles (later its O staging)
   static constexpr int kQBytes = 2 * kQBufBytes;        // double buffered across units
@@ -90,16 +90,21 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256u : 512u;
   static constexpr int kCtasPerSm = (kTmemCols == 256u) ? 2 : 1;
   // per-CTA shared-memory budget: the SM's 228 KB shared by kCtasPerSm CTAs,
-  // each also reserving 1 KB, minus the barrier block and alignment slack
-  static constexpr int kBudget = (228 * 1024) / kCtasPerSm - 1024 - kBarBytes - 1024;
+  // each also reserving 1 KB, minus the barrier block (the dynamic shared
+  // memory is declared 1024-byte aligned, so no alignment slack: at D = 128
+  // with two CTAs per SM that is what leaves room for a third ring stage)
+  static constexpr int kBudget = (228 * 1024) / kCtasPerSm - 1024 - kBarBytes;
   static constexpr int kStagesRaw = (kBudget - kQBytes) / kTileBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kRingBytes = kStages * kTileBytes;
   static constexpr int kBarOffset = kQBytes + kRingBytes;
-  static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;  // + barriers + alignment slack
+  static constexpr int kSmemBytes = kBarOffset + kBarBytes;
   static constexpr uint32_t kSCol(int w, int buf) { return static_cast<uint32_t>((kSBuf * w + buf) * BN); }
   static constexpr uint32_t kOCol(int w) { return static_cast<uint32_t>(kSBuf * NH * BN + w * D); }
   static_assert(kStages >= 2, "need at least two ring stages");
+  // full/empty per stage, q_full/q_empty [2], s_full/p_full [NH][2],
+  // pv_done/o_full/o_drained [NH], mma_done; then the TMEM base and the abort flag
+  static_assert((2 * kStages + 4 + 7 * NH + 1) * 8 + 8 <= kBarBytes, "barrier block");
   static_assert(kColsUsed <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared-memory budget");
 };
@@ -354,9 +359,15 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const Params p) {
   using C = Cfg<D, BN, NH>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // (128-byte swizzled tiles need 1024-byte aligned addresses; the budget
+  // has no slack for aligning by hand, so a base off the declared alignment
+  // is reported and nothing runs)
+  if (reinterpret_cast<uintptr_t>(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) report_launch_error(p.status, kWhereAlign);
+    return;
+  }
+  uint8_t *smem = smem_raw;
   uint8_t *sQ = smem;                       // [2] units' Q tiles, later their O staging
   uint8_t *sRing = smem + C::kQBytes;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);

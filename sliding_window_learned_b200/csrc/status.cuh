@@ -8,8 +8,9 @@ namespace attnsink {
 // up, records ATTN_ETIMEOUT and returns (1 s; a healthy wait is microseconds).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-// Must match ATTN_ETIMEOUT in include/attnsink.h.
+// Must match ATTN_ETIMEOUT and ATTN_ECUDA in include/attnsink.h.
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusCuda = -3;
 
 // Per-CTA context for bounded waits: a shared abort flag (so one timed-out
 // wait stops the whole CTA promptly) and the global status word
@@ -31,6 +32,12 @@ __device__ __forceinline__ uint64_t wait_limit_ns(const int *status) {
 
 __device__ __forceinline__ void report_timeout(int *status, int where) {
   if (atomicCAS(status, 0, kStatusTimeout) == 0) atomicExch(status + 1, where);
+}
+
+// A kernel that finds its launch unusable (dynamic shared memory not at the
+// alignment it declares) records ATTN_ECUDA and returns before any other work.
+__device__ __forceinline__ void report_launch_error(int *status, int where) {
+  if (atomicCAS(status, 0, kStatusCuda) == 0) atomicExch(status + 1, where);
 }
 
 }  // namespace attnsink
