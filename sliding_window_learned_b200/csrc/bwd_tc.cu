@@ -33,8 +33,10 @@
 //              one TMA bulk reduction per step; at a unit's end dK, dV (rows)
 //   warp 12    producer: K, V per unit, Q, dO per step (TMA, a ring of
 //              kStages slots) and the step's LSE and Dsum rows
-//   warp 13    TMEM allocation and the MMA issue (one thread)
-//   warps 14-15 idle (they pad the fourth warpgroup)
+//   warp 13    TMEM allocation and the issue of S^T, dP^T (one thread)
+//   warp 14    the issue of dV, dK and dQ^T (one thread): two issuers, so
+//              that neither group of products waits behind the other's issue
+//   warp 15    idle (it pads the fourth warpgroup)
 // dK and dV are summed over the units of a kv head in fp32 workspaces
 // (atomic adds), converted to bf16 afterwards like dQ.  Every wait is
 // bounded; a timeout records ATTN_ETIMEOUT and every role returns.
@@ -53,8 +55,8 @@ namespace {
 constexpr int kBK = 128;                        // keys per unit (TMEM lanes)
 constexpr int kBQ = 64;                         // queries per step
 constexpr int kThreads = 512;
-constexpr int kProducerWarp = 12, kMmaWarp = 13;
-constexpr uint32_t kTmemThreads = 416;          // warps 0-11 and the MMA warp
+constexpr int kProducerWarp = 12, kMmaWarp = 13, kMmaWarp2 = 14;
+constexpr uint32_t kTmemThreads = 448;          // warps 0-11 and the two MMA warps
 // Registers after reallocation: the two P^T/dS^T warpgroups hand some to the
 // producer/MMA warpgroup; the drain warpgroup keeps the launch value.
 constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8, kRegsSoftmax = 120, kRegsDrain = kRegsLaunch,
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *dsm_free = dq_empty + 1;     // [2] a step's dQ^T product read its dS^T tile
   uint64_t *dkv_full = dsm_free + 2;     // a unit's last dV, dK products finished
   uint64_t *dkv_free = dkv_full + 1;     // ... and dK, dV read out of TMEM (128)
-  uint64_t *mma_done = dkv_free + 1;     // every product of the CTA finished
+  uint64_t *mma_done = dkv_free + 1;     // every product of the CTA finished (both issuers)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   const WaitCtx ctx{abort_flag, p.status, wait_limit_ns(p.status)};
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
     mbar_init(dkv_free, 128);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   uint32_t tmem = 0;
-  const bool tmem_warp = warp < 12 || warp == kMmaWarp;
+  const bool tmem_warp = warp < 12 || warp == kMmaWarp || warp == kMmaWarp2;
   if (tmem_warp) {
     tc_fence_before();
     named_barrier_sync(kBarTmem, kTmemThreads);
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(kBK, kBQ, 0, 0);    // K-major A and B
@@ -320,98 +322,103 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t km_lo = umma_desc_lo(smem_u32(sK), kBK * 128);     // K as an M-major A
       const uint32_t ds_lo = umma_desc_lo(smem_u32(sDS), kBK * 128);    // dS^T as an N-major B
       bool ok = true;
-      struct Pending {
-        int g, slot, kvb, ul;
-        bool first, last;
-      };
-      Pending pend{0, 0, 0, 0, false, false};
-      bool have = false;
-      // the second half of a step: dV, dK once P^T, dS^T are in, then dQ^T
-      auto finish = [&](const Pending &r) -> bool {
-        if (!mbar_wait(p_full, static_cast<uint32_t>(r.g) & 1u, ctx, kWhereP)) return false;
-        // the first step of a unit overwrites dK, dV: the previous unit's
-        // must have been read out of TMEM
-        if (r.first && r.ul > 0 && !mbar_wait(dkv_free, static_cast<uint32_t>(r.ul - 1) & 1u, ctx, kWhereDkv))
-          return false;
-        tc_fence_after();
-        const uint32_t acc0 = r.first ? 0u : 1u;
-#pragma unroll
-        for (int kk = 0; kk < kBQ / 16; ++kk)
-          umma_ts_w(tmem + C::kColDV, tmem + kColP + kk * 8, don_lo + ((r.slot * C::kQTile + kk * 16 * 128) >> 4), hi,
-                    idesc_kv, kk > 0 ? 1u : acc0);
-#pragma unroll
-        for (int kk = 0; kk < kBQ / 16; ++kk)
-          umma_ts_w(tmem + C::kColDK, tmem + kColDS + kk * 8, qn_lo + ((r.slot * C::kQTile + kk * 16 * 128) >> 4), hi,
-                    idesc_kv, kk > 0 ? 1u : acc0);
-        umma_commit(pbuf_free);
-        umma_commit(&empty[r.slot]);
-        if (r.last) umma_commit(dkv_full);
-        // dQ^T overwrites the previous step's, which must have been read out
-        if (r.g > 0 && !mbar_wait(dq_empty, static_cast<uint32_t>(r.g - 1) & 1u, ctx, kWhereDq)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          umma_ss_w(tmem + C::kColDQ, km_lo + ((r.kvb * C::kKVTile + kk * 16 * 128) >> 4), hi,
-                    ds_lo + (((r.g & 1) * kDSTile + kk * 16 * 128) >> 4), hi, idesc_dq, kk > 0 ? 1u : 0u);
-        umma_commit(dq_full);
-        umma_commit(&dsm_free[r.g & 1]);
-        if (r.last) umma_commit(&kv_empty[r.kvb]);
-        return true;
-      };
       int g = 0, ul = 0;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
-        const Unit t = unit_at(p, u);
-        const int kvb = ul % kKVBuf;
-        // with one K/V buffer the previous unit must let go of it first
-        if (kKVBuf == 1 && have) {
-          have = false;
-          if (!finish(pend)) {
+      if (warp == kMmaWarp) {
+        // S^T = K Q^T and dP^T = V dO^T per step, once the softmax warps have
+        // read the previous step's out of TMEM
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
+          const Unit t = unit_at(p, u);
+          const int kvb = ul % kKVBuf;
+          if (!mbar_wait(&kv_full[kvb], static_cast<uint32_t>(ul / kKVBuf) & 1u, ctx, kWhereKv)) {
             ok = false;
             break;
+          }
+          const int steps = t.nh * t.nq;
+          for (int s = 0; s < steps; ++s, ++g) {
+            const int slot = g % kStages;
+            if (!mbar_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull)) {
+              ok = false;
+              break;
+            }
+            if (g > 0 && !mbar_wait(s_free, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereS)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
+              const uint32_t ka = ((kvb * C::kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
+              const uint32_t qa = ((slot * C::kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
+              umma_ss_w(tmem + kColS, k_lo + ka, hi, q_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t ka = ((kvb * C::kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
+              const uint32_t qa = ((slot * C::kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
+              umma_ss_w(tmem + kColDP, v_lo + ka, hi, do_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(s_full);
           }
         }
-        if (!mbar_wait(&kv_full[kvb], static_cast<uint32_t>(ul / kKVBuf) & 1u, ctx, kWhereKv)) {
-          ok = false;
-          break;
-        }
-        const int steps = t.nh * t.nq;
-        for (int s = 0; s < steps; ++s, ++g) {
-          const int slot = g % kStages;
-          if (!mbar_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull)) {
-            ok = false;
-            break;
-          }
-          // S^T and dP^T overwrite the previous step's, which the softmax
-          // warps must have read out
-          if (g > 0 && !mbar_wait(s_free, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereS)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+      } else {
+        // dV += P^T dO and dK += dS^T Q once P^T, dS^T of the step are in,
+        // then dQ^T = K^T dS^T.  (The step's Q, dO and the unit's K, V
+        // landed before the S^T product that led to P^T; the waits below
+        // are already complete and only order this thread after the copies.
+        // The S^T, dP^T products that read a slot or the K/V buffer finished
+        // before the softmax read S^T, so the releases committed here follow
+        // them.)
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
+          const Unit t = unit_at(p, u);
+          const int kvb = ul % kKVBuf;
+          const int steps = t.nh * t.nq;
+          for (int s = 0; s < steps; ++s, ++g) {
+            const int slot = g % kStages;
+            const bool first = s == 0, last = s == steps - 1;
+            if (!mbar_wait(p_full, static_cast<uint32_t>(g) & 1u, ctx, kWhereP) ||
+                !mbar_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull) ||
+                (first && !mbar_wait(&kv_full[kvb], static_cast<uint32_t>(ul / kKVBuf) & 1u, ctx, kWhereKv))) {
+              ok = false;
+              break;
+            }
+            // the first step of a unit overwrites dK, dV: the previous unit's
+            // must have been read out of TMEM
+            if (first && ul > 0 && !mbar_wait(dkv_free, static_cast<uint32_t>(ul - 1) & 1u, ctx, kWhereDkv)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // 16 channels = 32 bytes along the swizzled row; 64-channel chunks apart
-            const uint32_t ka = ((kvb * C::kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
-            const uint32_t qa = ((slot * C::kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
-            umma_ss_w(tmem + kColS, k_lo + ka, hi, q_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
-          }
+            for (int kk = 0; kk < kBQ / 16; ++kk)
+              umma_ts_w(tmem + C::kColDV, tmem + kColP + kk * 8, don_lo + ((slot * C::kQTile + kk * 16 * 128) >> 4),
+                        hi, idesc_kv, kk > 0 ? 1u : acc0);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = ((kvb * C::kKVTile + (kk >> 2) * kBK * 128) >> 4) + (kk & 3) * 2;
-            const uint32_t qa = ((slot * C::kQTile + (kk >> 2) * kBQ * 128) >> 4) + (kk & 3) * 2;
-            umma_ss_w(tmem + kColDP, v_lo + ka, hi, do_lo + qa, hi, idesc_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kBQ / 16; ++kk)
+              umma_ts_w(tmem + C::kColDK, tmem + kColDS + kk * 8, qn_lo + ((slot * C::kQTile + kk * 16 * 128) >> 4),
+                        hi, idesc_kv, kk > 0 ? 1u : acc0);
+            umma_commit(pbuf_free);
+            umma_commit(&empty[slot]);
+            if (last) umma_commit(dkv_full);
+            // dQ^T overwrites the previous step's, which must have been read out
+            if (g > 0 && !mbar_wait(dq_empty, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereDq)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              umma_ss_w(tmem + C::kColDQ, km_lo + ((kvb * C::kKVTile + kk * 16 * 128) >> 4), hi,
+                        ds_lo + (((g & 1) * kDSTile + kk * 16 * 128) >> 4), hi, idesc_dq, kk > 0 ? 1u : 0u);
+            umma_commit(dq_full);
+            umma_commit(&dsm_free[g & 1]);
+            if (last) umma_commit(&kv_empty[kvb]);
           }
-          umma_commit(s_full);
-          if (have && !finish(pend)) {
-            ok = false;
-            break;
-          }
-          pend = Pending{g, slot, kvb, ul, s == 0, s == steps - 1};
-          have = true;
         }
       }
-      if (ok && have) finish(pend);
-      // Every tensor-core operation of this CTA has finished before teardown.
+      // Every tensor-core operation of this CTA has finished before teardown
+      // (both issuers arrive).
       umma_commit(mma_done);
       drain_wait(mma_done, 0);
     }
