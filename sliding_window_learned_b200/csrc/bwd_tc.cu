@@ -34,9 +34,9 @@
 //   warp 12    producer: K, V per unit, Q, dO per step (TMA, a ring of
 //              kStages slots) and the step's LSE and Dsum rows
 //   warp 13    TMEM allocation and the issue of S^T, dP^T (one thread)
-//   warp 14    the issue of dV, dK and dQ^T (one thread): two issuers, so
-//              that neither group of products waits behind the other's issue
-//   warp 15    idle (it pads the fourth warpgroup)
+//   warp 14    the issue of dV, dK (one thread)
+//   warp 15    the issue of dQ^T (one thread): three issuers, so that no
+//              group of products waits behind another's issue
 // dK and dV are summed over the units of a kv head in fp32 workspaces
 // (atomic adds), converted to bf16 afterwards like dQ.  Every wait is
 // bounded; a timeout records ATTN_ETIMEOUT and every role returns.
@@ -55,8 +55,8 @@ namespace {
 constexpr int kBK = 128;                        // keys per unit (TMEM lanes)
 constexpr int kBQ = 64;                         // queries per step
 constexpr int kThreads = 512;
-constexpr int kProducerWarp = 12, kMmaWarp = 13, kMmaWarp2 = 14;
-constexpr uint32_t kTmemThreads = 448;          // warps 0-11 and the two MMA warps
+constexpr int kProducerWarp = 12, kMmaWarp = 13, kMmaWarp2 = 14, kMmaWarp3 = 15;
+constexpr uint32_t kTmemThreads = 480;          // warps 0-11 and the three MMA warps
 // Registers after reallocation: the two P^T/dS^T warpgroups hand some to the
 // producer/MMA warpgroup; the drain warpgroup keeps the launch value.
 constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8, kRegsSoftmax = 120, kRegsDrain = kRegsLaunch,
@@ -179,8 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *dsm_free = dq_empty + 1;     // [2] a step's dQ^T product read its dS^T tile
   uint64_t *dkv_full = dsm_free + 2;     // a unit's last dV, dK products finished
   uint64_t *dkv_free = dkv_full + 1;     // ... and dK, dV read out of TMEM (128)
-  uint64_t *mma_done = dkv_free + 1;     // every product of the CTA finished (both issuers)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  uint64_t *mma_done = dkv_free + 1;     // every product of the CTA finished (all three issuers)
+  // [2] dS^T of step g in shared memory (256), for the dQ^T issuer: one per
+  // dS^T buffer, so that each advances once every two steps and the softmax,
+  // which the dS^T buffers let run at most two steps ahead of that issuer,
+  // cannot bring a barrier back to the parity it waits for
+  uint64_t *dsp_full = mma_done + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dsp_full + 2);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   const WaitCtx ctx{abort_flag, p.status, wait_limit_ns(p.status)};
 
@@ -205,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
     mbar_init(dkv_free, 128);
-    mbar_init(mma_done, 2);
+    mbar_init(mma_done, 3);
+    for (int i = 0; i < 2; ++i) mbar_init(&dsp_full[i], 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -217,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   uint32_t tmem = 0;
-  const bool tmem_warp = warp < 12 || warp == kMmaWarp || warp == kMmaWarp2;
+  const bool tmem_warp = warp < 12 || warp == kMmaWarp || warp == kMmaWarp2 || warp == kMmaWarp3;
   if (tmem_warp) {
     tc_fence_before();
     named_barrier_sync(kBarTmem, kTmemThreads);
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(&full[k % kStages], static_cast<uint32_t>(k / kStages) & 1u);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
+  } else if (warp == kMmaWarp || warp == kMmaWarp2 || warp == kMmaWarp3) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(kBK, kBQ, 0, 0);    // K-major A and B
@@ -361,24 +367,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(s_full);
           }
         }
-      } else {
-        // dV += P^T dO and dK += dS^T Q once P^T, dS^T of the step are in,
-        // then dQ^T = K^T dS^T.  (The step's Q, dO and the unit's K, V
-        // landed before the S^T product that led to P^T; the waits below
-        // are already complete and only order this thread after the copies.
-        // The S^T, dP^T products that read a slot or the K/V buffer finished
-        // before the softmax read S^T, so the releases committed here follow
-        // them.)
+      } else if (warp == kMmaWarp2) {
+        // dV += P^T dO and dK += dS^T Q once P^T, dS^T of the step are in.
+        // (The step's Q, dO landed before the S^T product that led to P^T;
+        // the wait below is already complete and only orders this thread
+        // after the copies.  The S^T, dP^T products that read the slot
+        // finished before the softmax read S^T, so the release committed here
+        // follows them.)
         for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
           const Unit t = unit_at(p, u);
-          const int kvb = ul % kKVBuf;
           const int steps = t.nh * t.nq;
           for (int s = 0; s < steps; ++s, ++g) {
             const int slot = g % kStages;
             const bool first = s == 0, last = s == steps - 1;
             if (!mbar_wait(p_full, static_cast<uint32_t>(g) & 1u, ctx, kWhereP) ||
-                !mbar_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull) ||
-                (first && !mbar_wait(&kv_full[kvb], static_cast<uint32_t>(ul / kKVBuf) & 1u, ctx, kWhereKv))) {
+                !mbar_wait(&full[slot], static_cast<uint32_t>(g / kStages) & 1u, ctx, kWhereFull)) {
               ok = false;
               break;
             }
@@ -401,8 +404,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(pbuf_free);
             umma_commit(&empty[slot]);
             if (last) umma_commit(dkv_full);
-            // dQ^T overwrites the previous step's, which must have been read out
-            if (g > 0 && !mbar_wait(dq_empty, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereDq)) {
+          }
+        }
+      } else {
+        // dQ^T = K^T dS^T once dS^T of the step is in shared memory and the
+        // previous dQ^T has been read out.  (The unit's K landed before its
+        // first S^T product; the K/V release committed here at a unit's end
+        // follows that unit's S^T, dP^T products, which finished before the
+        // softmax read them.)
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++ul) {
+          const Unit t = unit_at(p, u);
+          const int kvb = ul % kKVBuf;
+          const int steps = t.nh * t.nq;
+          for (int s = 0; s < steps; ++s, ++g) {
+            const bool first = s == 0, last = s == steps - 1;
+            if (!mbar_wait(&dsp_full[g & 1], static_cast<uint32_t>(g >> 1) & 1u, ctx, kWhereP) ||
+                (first && !mbar_wait(&kv_full[kvb], static_cast<uint32_t>(ul / kKVBuf) & 1u, ctx, kWhereKv)) ||
+                (g > 0 && !mbar_wait(dq_empty, static_cast<uint32_t>(g - 1) & 1u, ctx, kWhereDq))) {
               ok = false;
               break;
             }
@@ -418,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Every tensor-core operation of this CTA has finished before teardown
-      // (both issuers arrive).
+      // (every issuer arrives).
       umma_commit(mma_done);
       drain_wait(mma_done, 0);
     }
@@ -512,6 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();                     // dS^T visible to the tensor cores
         tc_fence_before();
         mbar_arrive(p_full);
+        mbar_arrive(&dsp_full[g & 1]);
       }
     }
   } else {
