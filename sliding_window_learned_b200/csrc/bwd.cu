@@ -16,8 +16,8 @@
 //
 // Launches: a row kernel forms Dsum (from O as given: bf16 or, for the exact
 // form, f32) and the sink gradient; the tensor-core main pass (bwd_tc.cu)
-// sums dQ, dK and dV in fp32 workspaces; conversion kernels write them as
-// bf16.
+// sums dQ, dK and dV in fp32 workspaces; one conversion kernel writes them
+// as bf16.
 #include <math.h>
 
 #include <type_traits>
@@ -128,14 +128,32 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const OT *o, const __nv_b
 // fp32 [B, L, H, D] accumulator -> strided bf16 (dQ; dK and dV after the
 // tensor-core main pass): one thread per 8 channels, two 16-byte loads and
 // one 16-byte store.
+// One fp32 accumulator and its strided bf16 destination.
+struct ConvertJob {
+  const float *acc;
+  __nv_bfloat16 *out;
+  uint32_t rows, H;
+  int64_t s0, s1, s2;
+};
+
+// dQ, dK and dV in one launch: the grid strides over the three jobs' 8-channel
+// pieces in turn.
 template <int D>
-__global__ void bwd_convert_kernel(const float *acc, __nv_bfloat16 *out, uint32_t rows, uint32_t H, uint32_t L,
-                                   int64_t s0, int64_t s1, int64_t s2) {
+__global__ void bwd_convert_kernel(const ConvertJob j0, const ConvertJob j1, const ConvertJob j2, uint32_t L) {
   constexpr uint32_t kPer = D / 8;
-  const uint64_t n = static_cast<uint64_t>(rows) * kPer;
+  const uint64_t n0 = static_cast<uint64_t>(j0.rows) * kPer, n1 = static_cast<uint64_t>(j1.rows) * kPer;
+  const uint64_t n = n0 + n1 + static_cast<uint64_t>(j2.rows) * kPer;
   for (uint64_t e = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
-    const uint32_t r = static_cast<uint32_t>(e / kPer), c = static_cast<uint32_t>(e % kPer) * 8;
+    // (the job's fields picked one by one, so that none is copied to memory)
+    const bool in0 = e < n0, in1 = !in0 && e < n0 + n1;
+    const uint64_t el = in0 ? e : (in1 ? e - n0 : e - n0 - n1);
+    const float *acc = in0 ? j0.acc : (in1 ? j1.acc : j2.acc);
+    __nv_bfloat16 *out = in0 ? j0.out : (in1 ? j1.out : j2.out);
+    const uint32_t H = in0 ? j0.H : (in1 ? j1.H : j2.H);
+    const int64_t s0 = in0 ? j0.s0 : (in1 ? j1.s0 : j2.s0), s1 = in0 ? j0.s1 : (in1 ? j1.s1 : j2.s1),
+                  s2 = in0 ? j0.s2 : (in1 ? j1.s2 : j2.s2);
+    const uint32_t r = static_cast<uint32_t>(el / kPer), c = static_cast<uint32_t>(el % kPer) * 8;
     const uint32_t h = r % H, bi = r / H;
     const uint32_t i = bi % L, b = bi / L;
     const float4 x = *reinterpret_cast<const float4 *>(acc + static_cast<uint64_t>(r) * D + c);
@@ -202,22 +220,21 @@ cudaError_t launch_bwd(const BwdArgs &a, void *workspace, cudaStream_t stream) {
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = launch_bwd_main_tc(a, dsum, dq_acc, dk_acc, dv_acc, stream)) != cudaSuccess) return e;
-  auto convert = [&](const float *acc, void *out, int H, const int64_t *s) {
-    const uint64_t rows64 = static_cast<uint64_t>(a.B) * a.L * H;
-    if (rows64 > 0xFFFFFFFFull) return cudaErrorInvalidValue;
-    const uint64_t n = rows64 * (a.D / 8);
-    const int blocks = static_cast<int>(n / 256 + 1 < 148 * 8 ? n / 256 + 1 : 148 * 8);
-    if (a.D == 128)
-      bwd_convert_kernel<128><<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(out),
-                                                          static_cast<uint32_t>(rows64), H, a.L, s[0], s[1], s[2]);
-    else
-      bwd_convert_kernel<64><<<blocks, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16 *>(out),
-                                                         static_cast<uint32_t>(rows64), H, a.L, s[0], s[1], s[2]);
-    return cudaGetLastError();
+  auto job = [&](const float *acc, void *out, int H, const int64_t *s) {
+    return ConvertJob{acc, static_cast<__nv_bfloat16 *>(out), static_cast<uint32_t>(static_cast<uint64_t>(a.B) * a.L * H),
+                      static_cast<uint32_t>(H), s[0], s[1], s[2]};
   };
-  if ((e = convert(dq_acc, a.dq, a.Hq, a.dq_s)) != cudaSuccess) return e;
-  if ((e = convert(dk_acc, a.dk, a.Hkv, a.dk_s)) != cudaSuccess) return e;
-  return convert(dv_acc, a.dv, a.Hkv, a.dv_s);
+  const uint64_t rows64 = static_cast<uint64_t>(a.B) * a.L * (a.Hq + 2 * a.Hkv);
+  if (rows64 > 0xFFFFFFFFull) return cudaErrorInvalidValue;
+  const uint64_t n = rows64 * (a.D / 8);
+  const int blocks = static_cast<int>(n / 256 + 1 < 148 * 8 ? n / 256 + 1 : 148 * 8);
+  const ConvertJob jq = job(dq_acc, a.dq, a.Hq, a.dq_s), jk = job(dk_acc, a.dk, a.Hkv, a.dk_s),
+                   jv = job(dv_acc, a.dv, a.Hkv, a.dv_s);
+  if (a.D == 128)
+    bwd_convert_kernel<128><<<blocks, 256, 0, stream>>>(jq, jk, jv, static_cast<uint32_t>(a.L));
+  else
+    bwd_convert_kernel<64><<<blocks, 256, 0, stream>>>(jq, jk, jv, static_cast<uint32_t>(a.L));
+  return cudaGetLastError();
 }
 
 }  // namespace attnsink
