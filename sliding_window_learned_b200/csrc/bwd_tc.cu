@@ -57,12 +57,9 @@ constexpr int kBQ = 64;                         // queries per step
 constexpr int kThreads = 512;
 constexpr int kProducerWarp = 12, kMmaWarp = 13, kMmaWarp2 = 14, kMmaWarp3 = 15;
 constexpr uint32_t kTmemThreads = 480;          // warps 0-11 and the three MMA warps
-// Registers after reallocation: the two P^T/dS^T warpgroups hand some to the
-// producer/MMA warpgroup; the drain warpgroup keeps the launch value.
-constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8, kRegsSoftmax = 120, kRegsDrain = kRegsLaunch,
-                   kRegsOther = 144;
-static_assert(128 * (2 * kRegsSoftmax + kRegsDrain + kRegsOther) <= kRegsLaunch * kThreads,
-              "register split exceeds the launch allocation");
+// Every warpgroup keeps the launch allocation (128 registers): handing some
+// of the P^T/dS^T warpgroups' registers to the producer/MMA warpgroup
+// measured 1-3 % slower (the exponentiation pass is latency-bound).
 constexpr uint32_t kBarTmem = 1, kBarDrain = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -231,7 +228,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem = *tmem_slot;
   }
   if (warp >= 12) {
-  setmaxnreg_inc<kRegsOther>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -445,7 +441,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 8) {
     // --------------- P^T, dS^T: one key row per thread, 32 query columns per
     // warpgroup (warpgroup 0 the first half of the step's queries)
-    setmaxnreg_dec<kRegsSoftmax>();
     const int r = threadIdx.x & 127;                  // key row == TMEM lane
     const int c0 = (warp >> 2) * 32;                  // this warpgroup's first column
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
