@@ -135,3 +135,23 @@ def test_bwd_strided_packed_qkv():
     assert swl.attn_sink_get_status() == 0
     got = [t.float().cpu().numpy() for t in (dq, dk, dv, dsink)]
     _check(got, ref, "strided bwd")
+
+
+@pytest.mark.parametrize("o_kind", ["f32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_bwd_o_rows_unaligned(o_kind, D):
+    """O given as a slice of a [B, L, Hq, D + 1] buffer: its row strides are odd,
+    so the row kernel takes its scalar loads (a 16-byte load there would be
+    misaligned)."""
+    B, L, Hq, Hkv, W = 1, 200, 4, 2, 70
+    q, k, v, do, s = _case(B, L, Hq, Hkv, D, seed=5 + D)
+    scale = 1.0 / np.sqrt(D)
+    ref = oracle.bwd(inputs.bits(q), inputs.bits(k), inputs.bits(v), s.numpy(), inputs.bits(do), W, scale)
+    dt = torch.float32 if o_kind == "f32" else torch.bfloat16
+    pad = torch.zeros(B, L, Hq, D + 1, dtype=dt, device=DEV)
+    o = pad[..., :D]
+    o.copy_(torch.from_numpy(ref[4]).to(dt))
+    assert o.stride(2) % 2 == 1 and not o.is_contiguous()
+    lse = torch.from_numpy(ref[5]).float()
+    got = _gpu_bwd(q, k, v, o, lse, do, s, W, scale)
+    _check(got, ref, f"bwd ({o_kind} O, odd strides)")
