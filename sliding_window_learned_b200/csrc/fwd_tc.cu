@@ -23,10 +23,12 @@
 //   4*NH         TMA producer: Q (NH tiles) once, then K_0, K_1, then V_j,
 //                K_{j+2} per tile (one S buffer: K_0, then V_j, K_{j+1})
 //                into a ring of shared-memory stages
-//   4*NH+1       TMEM allocator and MMA issuer: per key tile j and head w,
-//                PV^w_j then the S^w it frees a buffer for, so that the
-//                tensor cores compute one tile while the softmax works on
-//                another.
+//   4*NH+1+w     MMA issuer of head w (4*NH+1 also allocates TMEM): per key
+//                tile j, PV^w_j then the S^w it frees a buffer for, so that
+//                the tensor cores compute one tile while the softmax works on
+//                another.  One issuing thread per head: an issuing thread
+//                blocks while the tensor pipe accepts each instruction, so
+//                one head's issue never queues behind the other's.
 // TMEM (columns): S^w buffer b at (kSBuf*w + b)*BN (P^w written as bf16 over
 // its first BN/2 columns), O^w after all S buffers.
 // Only the K tiles that meet the window [m0-W+1, m0+127] are visited; the
@@ -62,7 +64,7 @@ template <int D, int BN, int NH>
 struct Cfg {
   static constexpr int kSoftmaxWarps = 4 * NH;
   static constexpr int kProducerWarp = 4 * NH;
-  static constexpr int kMmaWarp = 4 * NH + 1;
+  static constexpr int kMmaWarp = 4 * NH + 1;     // issuer of head w: kMmaWarp + w
   // With two softmax warpgroups the producer and MMA warps are padded to a
   // whole third warpgroup, which hands registers to the softmax warpgroups.
   static constexpr int kWarps = NH == 2 ? 12 : 4 * NH + 2;
@@ -74,7 +76,8 @@ struct Cfg {
   // The warps that touch TMEM: the softmax warpgroups and the MMA warp.  This
   // is the single definition of the TMEM allocation barrier's participant
   // set; the barrier count and the participation test both derive from it.
-  static constexpr uint32_t kTmemWarpMask = ((1u << (4 * NH)) - 1u) | (1u << kMmaWarp);
+  static constexpr uint32_t kTmemWarpMask = ((1u << (4 * NH)) - 1u) | (((1u << NH) - 1u) << kMmaWarp);
+  static_assert(kMmaWarp + NH <= kWarps, "issuer warps");
   static constexpr uint32_t kTmemThreads = 32u * __builtin_popcount(kTmemWarpMask);
 
   static constexpr int kChunks = D / 64;          // 64-channel (128-byte) column chunks
@@ -426,7 +429,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], NH);              // each head's issuer frees the stage
     }
     for (int qb = 0; qb < 2; ++qb) {
       mbar_init(&q_full[qb], 1);
@@ -441,7 +444,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
       mbar_init(&o_full[w], 1);
       mbar_init(&o_drained[w], 128);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, NH);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -539,8 +542,9 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         drain_wait(&full[t % C::kStages], static_cast<uint32_t>(t / C::kStages) & 1u);
     }
     __syncwarp();
-  } else if (warp == C::kMmaWarp) {
+  } else if (warp >= C::kMmaWarp && warp < C::kMmaWarp + NH) {
     // ----------------------------------------------------------------- MMA
+    const int w = warp - C::kMmaWarp;        // this warp issues head w's products
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(kBM, BN, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_pv = umma_idesc_bf16(kBM, D, 0, 1);   // V is N-major
@@ -611,7 +615,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
           tc_fence_after();
           for (int jj = 0; ok && jj < C::kSBuf && jj < t.n_tiles; ++jj) {
             if (!acquire(ks)) break;
-            for (int w = 0; w < NH; ++w) issue_s(w, ks, jg + jj, qb);
+            issue_s(w, ks, jg + jj, qb);
             umma_commit(&empty[ks]);
           }
         }
@@ -620,7 +624,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
           const bool more = j + C::kSBuf < t.n_tiles;
           const bool last = j == t.n_tiles - 1;
           if (!acquire(vs)) break;
-          for (int w = 0; w < NH; ++w) {
+          {
             if (!mbar_wait(&p_full[2 * w + g % C::kSBuf], static_cast<uint32_t>(g / C::kSBuf) & 1u,
                            ctx, kWhereP)) {
               ok = false;
@@ -636,22 +640,20 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
             tc_fence_after();
             issue_pv(w, vs, g, j);
             if (last) umma_commit(&o_full[w]);   // this unit's O^w is complete
-            if (w == NH - 1) umma_commit(&empty[vs]);
+            umma_commit(&empty[vs]);
             // the S that this PV frees the buffer for: this unit's S_{j+kSBuf},
             // or (one buffer, last tile) the next unit's S_0, global tile g + 1
             if (more || (last && early_next)) {
-              if (w == 0) {
-                if (!more) {
-                  if (!mbar_wait(&q_full[qb ^ 1], static_cast<uint32_t>((ul + 1) >> 1) & 1u, ctx, kWhereQ)) {
-                    ok = false;
-                    break;
-                  }
-                  tc_fence_after();
+              if (!more) {
+                if (!mbar_wait(&q_full[qb ^ 1], static_cast<uint32_t>((ul + 1) >> 1) & 1u, ctx, kWhereQ)) {
+                  ok = false;
+                  break;
                 }
-                if (!acquire(ks)) break;
+                tc_fence_after();
               }
+              if (!acquire(ks)) break;
               issue_s(w, ks, g + C::kSBuf, more ? qb : qb ^ 1);
-              if (w == NH - 1) umma_commit(&empty[ks]);
+              umma_commit(&empty[ks]);
             }
           }
         }
@@ -668,7 +670,7 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
     tc_fence_before();
     named_barrier_sync(kBarTmem, C::kTmemThreads);
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    if (warp == C::kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
   }
   } else {
     if constexpr (C::kRealloc) setmaxnreg_inc<C::kRegsSoftmax>();
