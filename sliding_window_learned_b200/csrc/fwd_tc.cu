@@ -16,8 +16,9 @@
 // kv-head group.  The dispatched form is NH = 1: one head per CTA, 64-key
 // tiles, two S buffers (S_{j+1} is computed while tile j is exponentiated),
 // 256 TMEM columns, so two CTAs share each SM and their MMA streams and
-// exponentials interleave.  (NH = 2, two heads of a group sharing each
-// 128-key K/V tile in one CTA, measured slower on every workload.)  Warps:
+// exponentials interleave.  (NH = 2, two heads of a group sharing each K/V
+// tile in one CTA, measured as fast at W = 513 and slower at full causal
+// with 64-key tiles, slower everywhere with 128-key tiles.)  Warps:
 //   0 .. 4*NH-1  softmax / correction / epilogue: warpgroup w owns head slot
 //                w, one thread per query row (TMEM lane)
 //   4*NH         TMA producer: Q (NH tiles) once, then K_0, K_1, then V_j,
@@ -915,9 +916,11 @@ cudaError_t launch_max_logit_init(float *ml, int64_t sb, int B, int Hq, cudaStre
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream) {
   // One query head per CTA, 64-key tiles with two S buffers, two CTAs per SM,
   // for every group size.  (The kernel also takes two query heads of a kv
-  // group per CTA, NH = 2, sharing each K/V tile; measured on B200 that was
-  // slower on every workload: W = 513 534 against 587 TFLOP/s, full causal
-  // 967 against 1051, packed sequences 7-11 % slower.)
+  // group per CTA, NH = 2, sharing each K/V tile.  Measured on B200: with
+  // 128-key tiles slower on every workload (W = 513 534 against 587 TFLOP/s,
+  // full causal 967 against 1051, packed sequences 7-11 % slower); with 64-key
+  // tiles and one issuer per head 612 against 615 at W = 513 and 916 against
+  // 1070 at full causal.)
   const bool packed = a.cu_seqlens != nullptr;
   const bool ml = a.max_logit != nullptr;   // (batched inputs only)
   if (packed && ml) return cudaErrorInvalidValue;
