@@ -28,7 +28,6 @@
 namespace attnsink {
 namespace {
 
-
 // ------------------------------------------------------------------ rows
 // Dsum[b, h, i] = dO . O for every row, and dsink[h] -= exp(sink - LSE) * Dsum
 // (one atomic per block).  A block takes kRowBlock rows of one (batch, head);
@@ -166,9 +165,9 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const OT *o, const __nv_b
 }
 
 // ------------------------------------------------------------------ dQ out
-// fp32 [B, L, H, D] accumulator -> strided bf16 (dQ; dK and dV after the
-// tensor-core main pass): one thread per 8 channels, two 16-byte loads and
-// one 16-byte store.
+// fp32 [B, L, H, D] accumulators -> strided bf16 (dQ; dK and dV after the
+// tensor-core main pass): per 8 channels two 16-byte loads and one 16-byte
+// store.
 // One fp32 accumulator and its strided bf16 destination.
 struct ConvertJob {
   const float *acc;
