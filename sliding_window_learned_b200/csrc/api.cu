@@ -872,7 +872,7 @@ int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor 
 
 int attn_sink_set_wait_limit_ns(uint64_t ns) {
   t_last_error[0] = '\0';
-  int *dptr;
+  int *dptr = nullptr;
   int rc = status_ptr(&dptr);
   if (rc) return rc;
   const unsigned long long v = ns;

@@ -45,7 +45,6 @@ namespace {
 constexpr int kTK = 64;               // keys per tile (bf16 cache)
 constexpr int kConsumerWarps = 4;     // each owns 16 keys of every tile (bf16 cache)
 
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 enum : int { kWhereFull = 201, kWhereEmpty = 202, kWhereMerge = 203 };
 

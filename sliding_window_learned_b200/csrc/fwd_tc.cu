@@ -160,17 +160,6 @@ __device__ __forceinline__ void mask_chunk(uint32_t (&x)[32], int c0, int lo, in
     if (c0 + t < lo || c0 + t > hi) x[t] = __float_as_uint(-INFINITY);
 }
 
-__device__ __forceinline__ float max32(const uint32_t (&x)[32]) {
-  float a[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) a[u] = __uint_as_float(x[u]);
-#pragma unroll
-  for (int t = 4; t < 32; t += 4)
-#pragma unroll
-    for (int u = 0; u < 4; ++u) a[u] = fmaxf(a[u], __uint_as_float(x[t + u]));
-  return fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
