@@ -5,7 +5,6 @@ Bar: max|dO| <= 2e-2 and max|dLSE| <= 1e-3 over every compared element, and no
 NaN/Inf anywhere in the outputs.  Output buffers sit inside NaN-filled guard
 bands that must come back untouched; inputs are views into larger NaN-filled
 storage, so a read past the end of a sequence would show up as NaN."""
-import math
 
 import numpy as np
 import pytest
