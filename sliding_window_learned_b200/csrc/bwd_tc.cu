@@ -41,6 +41,8 @@
 // (atomic adds), converted to bf16 afterwards like dQ.  Every wait is
 // bounded; a timeout records ATTN_ETIMEOUT and every role returns.
 #include <cuda.h>
+
+#include <algorithm>
 #include <math.h>
 
 #include <type_traits>
@@ -650,15 +652,29 @@ cudaError_t launch_tc(const BwdArgs &a, const float *dsum, float *dq_acc, float 
   p.W = a.W;
   p.G = a.Hq / a.Hkv;
   p.nkb = (a.L + kBK - 1) / kBK;
-  // Split each kv head's query heads over units until there are about four
-  // units per SM (whole heads per unit; the units of a kv head add their dK,
-  // dV into the same fp32 rows).
+  // Split each kv head's query heads over units (whole heads per unit; the
+  // units of a kv head add their dK, dV into the same fp32 rows): the fewest
+  // units whose largest is at most a fifth of an SM's average share of the
+  // steps.  The static schedule then ends within about that of the average,
+  // and every further unit costs a K/V load and a dK/dV write-out.  A key
+  // block kb sees query blocks 2 kb .. last(kb) / 64, last(kb) =
+  // min(L - 1, 128 kb + 127 + min(W - 1, L)); block 0 sees the most.
   const int64_t base = static_cast<int64_t>(p.nkb) * a.Hkv * a.B;
-  p.hsplit = 1;
+  const int64_t wc = a.W - 1 < a.L ? a.W - 1 : a.L;
+  const int64_t nq_int = (127 + wc) / 64 + 1;               // blocks whose window ends before L - 1
+  const int64_t k1 = a.L - 1 - 127 - wc >= 0
+                         ? std::min<int64_t>(p.nkb, (a.L - 1 - 127 - wc) / 128 + 1) : 0;
+  const int64_t qlast = (a.L - 1) / 64, ntail = p.nkb - k1;
+  const int64_t steps_per_head = k1 * nq_int + ntail * (qlast + 1) - (k1 + p.nkb - 1) * ntail;
+  const int64_t nq_max = std::min<int64_t>(a.L - 1, 127 + wc) / 64 + 1;
+  const int64_t total_steps = steps_per_head * a.Hq * a.B;
+  p.hsplit = p.G;
   for (int hs = 1; hs <= p.G; ++hs) {
     if (p.G % hs) continue;
-    p.hsplit = hs;
-    if (base * hs >= 4LL * sms) break;
+    if (base * hs >= sms && 5 * (p.G / hs) * nq_max * sms <= total_steps) {
+      p.hsplit = hs;
+      break;
+    }
   }
   const int64_t units = base * p.hsplit;
   if (units > (1LL << 30)) return cudaErrorInvalidValue;
