@@ -163,7 +163,9 @@ int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k,
  *   k, v        [B, L, Hkv, D] bf16
  *   o           [B, L, Hq, D]  the forward's output: bf16 (as attn_sink_fwd
  *               writes it; Dsum then carries its rounding) or f32 (Dsum exact,
- *               the form issue #2969 asks for)
+ *               the form issue #2969 asks for); any outer strides (read with
+ *               16-byte loads when they keep rows 16-byte aligned, else
+ *               element by element)
  *   lse         [B, Hq, L]     f32, the forward's log-sum-exp (sink included)
  *   sinks, window, scale: as for attn_sink_fwd.
  *   dq          [B, L, Hq, D]  bf16, written completely
@@ -175,8 +177,8 @@ int attn_sink_fwd_cudacore(const attn_tensor *q, const attn_tensor *k,
  * accumulators, 2*B*L*Hkv*D*4 bytes.  The main pass runs on the
  * 5th-generation tensor cores (tcgen05, TMEM accumulators), accumulating in
  * fp32 with P and dS rounded to bf16 for the products.  Launches: a row
- * kernel, the main pass, then the fp32 -> bf16 conversions; no host
- * synchronisation.
+ * kernel (Dsum, the sink gradient, zeroed accumulators), the main pass, then
+ * one fp32 -> bf16 conversion of dq, dk and dv; no host synchronisation.
  */
 int attn_sink_bwd(const attn_tensor *q, const attn_tensor *k, const attn_tensor *v,
                   const attn_tensor *o, const attn_tensor *lse, const attn_tensor *dout,
