@@ -12,26 +12,23 @@
 // two query tiles per CTA in ping-pong) as prior art; everything here is
 // written for sm_100a directly.
 //
-// One CTA computes one 128-row query tile for NH query heads of the same
-// kv-head group.  The dispatched form is NH = 1: one head per CTA, 64-key
-// tiles, two S buffers (S_{j+1} is computed while tile j is exponentiated),
-// 256 TMEM columns, so two CTAs share each SM and their MMA streams and
-// exponentials interleave.  (NH = 2, two heads of a group sharing each K/V
-// tile in one CTA, measured as fast at W = 513 and slower at full causal
-// with 64-key tiles, slower everywhere with 128-key tiles.)  Warps:
-//   0 .. 4*NH-1  softmax / correction / epilogue: warpgroup w owns head slot
-//                w, one thread per query row (TMEM lane)
-//   4*NH         TMA producer: Q (NH tiles) once, then K_0, K_1, then V_j,
-//                K_{j+2} per tile (one S buffer: K_0, then V_j, K_{j+1})
-//                into a ring of shared-memory stages
-//   4*NH+1+w     MMA issuer of head w (4*NH+1 also allocates TMEM): per key
-//                tile j, PV^w_j then the S^w it frees a buffer for, so that
-//                the tensor cores compute one tile while the softmax works on
-//                another.  One issuing thread per head: an issuing thread
-//                blocks while the tensor pipe accepts each instruction, so
-//                one head's issue never queues behind the other's.
-// TMEM (columns): S^w buffer b at (kSBuf*w + b)*BN (P^w written as bf16 over
-// its first BN/2 columns), O^w after all S buffers.
+// One CTA computes one 128-row query tile of one query head: 64-key tiles,
+// two S buffers (S_{j+1} is computed while tile j is exponentiated), 256 TMEM
+// columns at D <= 128, so two CTAs share each SM and their MMA streams and
+// exponentials interleave (one CTA per SM at D = 256).  (Two heads of a kv
+// group per CTA, sharing each K/V tile, measured as fast at W = 513 and
+// slower at full causal with 64-key tiles and one MMA issuer per head, and
+// slower everywhere with 128-key tiles.)  Warps (the head slot w is 0; the
+// indexing is written per head):
+//   0 .. 3       softmax / correction / epilogue, one thread per query row
+//                (TMEM lane)
+//   4            TMA producer: Q once per unit, then K_0, K_1, then V_j,
+//                K_{j+2} per tile into a ring of shared-memory stages
+//   5            TMEM allocator and MMA issuer: per key tile j, PV_j then the
+//                S it frees a buffer for, so that the tensor cores compute
+//                one tile while the softmax works on another.
+// TMEM (columns): S buffer b at b*BN (P written as bf16 over its first BN/2
+// columns), O after both S buffers.
 // Only the K tiles that meet the window [m0-W+1, m0+127] are visited; the
 // mask is applied on the tiles that cross the causal diagonal, the window's
 // lower edge or the end of the sequence.
@@ -66,14 +63,12 @@ struct Cfg {
   static constexpr int kSoftmaxWarps = 4 * NH;
   static constexpr int kProducerWarp = 4 * NH;
   static constexpr int kMmaWarp = 4 * NH + 1;     // issuer of head w: kMmaWarp + w
-  // With two softmax warpgroups the producer and MMA warps are padded to a
-  // whole third warpgroup, which hands registers to the softmax warpgroups.
-  static constexpr int kWarps = NH == 2 ? 12 : 4 * NH + 2;
+  static constexpr int kWarps = 4 * NH + 2;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr bool kRealloc = NH == 2;
-  static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
-  static_assert(!kRealloc || (8 * kRegsSoftmax + 4 * kRegsOther) * 32 <= 65536 / kThreads / 8 * 8 * kThreads,
-                "register split exceeds the launch allocation");
+  // (The head-slot indexing below is written for NH heads per CTA; one is
+  // built.  Two heads per CTA, with 64- and 128-key tiles, were measured with
+  // earlier versions of this kernel and were slower or no faster.)
+  static_assert(NH == 1, "one query head per CTA");
   // The warps that touch TMEM: the softmax warpgroups and the MMA warp.  This
   // is the single definition of the TMEM allocation barrier's participant
   // set; the barrier count and the participation test both derive from it.
@@ -87,9 +82,8 @@ struct Cfg {
   static constexpr int kQBufBytes = NH * kQTileBytes;   // one unit's Q tiles (later its O staging)
   static constexpr int kQBytes = 2 * kQBufBytes;        // double buffered across units
   static constexpr int kTileBytes = BN * D * 2;   // one K or V tile
-  // S buffers per head: two (S_{j+1} computed while S_j is exponentiated)
-  // when TMEM has room, else one (the other head's work fills the gap)
-  static constexpr int kSBuf = NH * (2 * BN + D) <= 512 ? 2 : 1;
+  // two S buffers: S_{j+1} is computed while S_j is exponentiated
+  static constexpr int kSBuf = 2;
   static constexpr int kColsUsed = NH * (kSBuf * BN + D);
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256u : 512u;
   static constexpr int kCtasPerSm = (kTmemCols == 256u) ? 2 : 1;
@@ -456,9 +450,6 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
   }
 
   if (warp >= C::kSoftmaxWarps) {
-  // Producer/MMA warpgroup: hand registers to the softmax warpgroups (every
-  // warp of the warpgroup, the idle padding warps included, executes this).
-  if constexpr (C::kRealloc) setmaxnreg_dec<C::kRegsOther>();
   if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -584,20 +575,12 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         umma_commit(&pv_done[w]);
       };
       int jg = 0;                            // tiles of earlier units (barrier phases)
-      bool pre = false;                      // this unit's first S (every head) already issued
       for (int ul = 0, u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const Unit t = unit_at(u);
         if (packed && t.n_tiles <= 0) continue;   // ul counts the units that are not empty
         const int qb = ul & 1;
-        // With one S buffer per head, the next unit's first S^w is issued
-        // right behind this unit's last PV^w, so that it is ready when the
-        // warpgroup finishes this unit's epilogue.
-        int un = u + static_cast<int>(gridDim.x);
-        if constexpr (packed)
-          while (un < p.num_units && unit_at(un).n_tiles <= 0) un += gridDim.x;
-        const bool early_next = C::kSBuf == 1 && un < p.num_units;
         int ks = 0, vs = 0;
-        if (!pre) {
+        {
           if (!mbar_wait(&q_full[qb], static_cast<uint32_t>(ul >> 1) & 1u, ctx, kWhereQ)) {
             ok = false;
             break;
@@ -631,23 +614,14 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
             issue_pv(w, vs, g, j);
             if (last) umma_commit(&o_full[w]);   // this unit's O^w is complete
             umma_commit(&empty[vs]);
-            // the S that this PV frees the buffer for: this unit's S_{j+kSBuf},
-            // or (one buffer, last tile) the next unit's S_0, global tile g + 1
-            if (more || (last && early_next)) {
-              if (!more) {
-                if (!mbar_wait(&q_full[qb ^ 1], static_cast<uint32_t>((ul + 1) >> 1) & 1u, ctx, kWhereQ)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-              }
+            // the S that this PV frees the buffer for: S_{j+kSBuf}
+            if (more) {
               if (!acquire(ks)) break;
-              issue_s(w, ks, g + C::kSBuf, more ? qb : qb ^ 1);
+              issue_s(w, ks, g + C::kSBuf, qb);
               umma_commit(&empty[ks]);
             }
           }
         }
-        pre = early_next;
         jg += t.n_tiles;
         ++ul;
       }
@@ -663,7 +637,6 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
     if (warp == C::kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
   }
   } else {
-    if constexpr (C::kRealloc) setmaxnreg_inc<C::kRegsSoftmax>();
     // ------------------------------------------- softmax / correction / epilogue
     const int w = warp >> 2;                         // head slot of this warpgroup
     const int r = threadIdx.x & 127;                 // tile row == TMEM lane
@@ -776,29 +749,13 @@ __global__ void __launch_bounds__(Cfg<D, BN, NH>::kThreads, Cfg<D, BN, NH>::kCta
         }
       };
       static_assert(D % 64 == 0, "chunks are converted in pairs");
-      if constexpr (packed || NH == 1) {
-        // (the packed kernel keeps one chunk in flight: its row-by-row stores
-        // leave no registers for a second; so does the one-head kernel, which
-        // has no register reallocation and measured 1.6 % slower with two)
+      // one chunk in flight (two measured 1.6 % slower: registers)
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + o_col + c * 32, o);
-          tmem_wait_ld_dep(o);
-          convert(c, o);
-        }
-      } else {
-        uint32_t oa[32], ob[32];
-        tmem_ld32(lane_base + o_col, oa);
-#pragma unroll
-        for (int c = 0; c < D / 32; c += 2) {
-          tmem_wait_ld_dep(oa);
-          tmem_ld32(lane_base + o_col + (c + 1) * 32, ob);
-          convert(c, oa);
-          tmem_wait_ld_dep(ob);
-          if (c + 2 < D / 32) tmem_ld32(lane_base + o_col + (c + 2) * 32, oa);
-          convert(c + 1, ob);
-        }
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + o_col + c * 32, o);
+        tmem_wait_ld_dep(o);
+        convert(c, o);
       }
       tc_fence_before();
       mbar_arrive(&o_drained[w]);
@@ -903,13 +860,8 @@ cudaError_t launch_max_logit_init(float *ml, int64_t sb, int B, int Hq, cudaStre
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs &a, cudaStream_t stream) {
-  // One query head per CTA, 64-key tiles with two S buffers, two CTAs per SM,
-  // for every group size.  (The kernel also takes two query heads of a kv
-  // group per CTA, NH = 2, sharing each K/V tile.  Measured on B200: with
-  // 128-key tiles slower on every workload (W = 513 534 against 587 TFLOP/s,
-  // full causal 967 against 1051, packed sequences 7-11 % slower); with 64-key
-  // tiles and one issuer per head 612 against 615 at W = 513 and 916 against
-  // 1070 at full causal.)
+  // One query head per CTA, 64-key tiles with two S buffers, two CTAs per SM
+  // (one at D = 256), for every group size.
   const bool packed = a.cu_seqlens != nullptr;
   const bool ml = a.max_logit != nullptr;   // (batched inputs only)
   if (packed && ml) return cudaErrorInvalidValue;
